@@ -1,0 +1,307 @@
+"""CPU oracle for the Sparse-BitLinear operator (test infrastructure).
+
+This module is test infrastructure.  Only the tests under ``tests/``,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import or call it.  The CUDA library
+(``semi_structured_sparsity_step_b200``) never imports it, and it imports
+nothing from the CUDA library: the two share no code.  Inputs come from the
+seeded generators in ``synth`` as raw bf16 bit patterns (numpy ``uint16``).
+
+It is a plain, slow restatement of what the operator computes, written in
+numpy so that each step can be checked against the pages by eye.  Floating
+point steps that decide integers (ternary codes, int8 activations) are
+written as explicit IEEE fp32 operations, in the order given below, so that
+a GPU implementation can reproduce them bit for bit; the reductions that only
+feed float outputs (the backward products) are done in fp64.
+
+Pages cited (titles as they appear on the pages):
+
+* [summary]   "Sparse-BitNet：1.58-bit 大模型天然兼容半结构化稀疏" -- the
+  structured summary of arXiv 2603.05168 (sections 前置知识, 核心方法,
+  方法步骤详情 / Algorithm 1, 局限与改进, 独立分析的弱点, 论文图表).
+* [gist]      the gist.science technical summary of the same paper
+  (section 2.2 "Sparse-BitNet 框架").
+* [explainer] "什麼是 Sparse-BitNet？核心概念一次搞懂" (sections
+  "1.58 位元量化的技術原理", "N:M 半結構化稀疏性的運作機制").
+* [article]   "突破性发现：极低位量化与稀疏化的完美协同" (section 7.1,
+  "推理优化技巧").
+
+Readings taken where the pages are silent (each is pinned by a test):
+
+* ties in |W| inside a group go to the lowest index;
+* the quantiser divides by (gamma + 1e-5); outputs are scaled by gamma;
+* gamma is the exact mean of |W| over the whole tensor, rounded once to
+  fp64 (correctly rounded sum, then an fp64 division), then to fp32;
+* an all-zero activation row uses max|x| = 1e-5 (so it quantises to zeros);
+* the straight-through estimator is the identity through the activation
+  quantiser, RoundClip and the N:M selector; no gradient flows through gamma.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(none is "parity unpinned").
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+EPS = np.float32(1e-5)          # quantiser epsilon (denominator only)
+ACT_FLOOR = np.float32(1e-5)    # floor for max|x| of a token
+QMAX = np.float32(127.0)        # int8 absmax level
+
+
+# --------------------------------------------------------------------------
+# bf16 decoding (format plumbing, exact)
+# --------------------------------------------------------------------------
+def bf16_to_f32(u16: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> the same values as fp32 (exact widening)."""
+    u16 = np.ascontiguousarray(u16, dtype=np.uint16)
+    return (u16.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+# --------------------------------------------------------------------------
+# (a1) N:M magnitude mask  M_{N:M} = Pi_{N:M}(|W|)
+# [summary] 半结构化 N:M 稀疏 (||M_group||_0 = N per M consecutive weights);
+# [summary] 核心方法 (i) and Algorithm 1 step (2): top-N by magnitude of the
+# continuous master weight, recomputed every step; [gist] 2.2 (mask from
+# master weights, not from ternary weights).
+# --------------------------------------------------------------------------
+def nm_mask(w_bits: np.ndarray, N: int, M: int, chunk: int = 1 << 18) -> np.ndarray:
+    """Keep-mask (bool, same shape as W): top-N of |W| in each group of M
+    consecutive weights along d_in.
+
+    Rank of position j in its group: the number of members with a strictly
+    larger magnitude plus the number of earlier members with an equal one.
+    Position j is kept iff rank_j < N.  This keeps exactly N per group and
+    breaks ties toward the lowest index.
+    """
+    d_out, d_in = w_bits.shape
+    assert d_in % M == 0 and 1 <= N <= M
+    a_all = np.abs(bf16_to_f32(w_bits)).reshape(-1, M)
+    earlier = np.tri(M, k=-1, dtype=bool)          # earlier[j, k] = (k < j)
+    keep = np.empty(a_all.shape, dtype=bool)
+    for s in range(0, a_all.shape[0], chunk):
+        a = a_all[s:s + chunk]
+        aj = a[:, :, None]
+        ak = a[:, None, :]
+        rank = (ak > aj).sum(axis=2) + ((ak == aj) & earlier).sum(axis=2)
+        keep[s:s + chunk] = rank < N
+    return keep.reshape(d_out, d_in)
+
+
+# --------------------------------------------------------------------------
+# (a2) absmean scale  gamma = ||W||_1 / (d_out * d_in)
+# [summary] 前置知识, "1.58-bit BitNet 量化".
+# --------------------------------------------------------------------------
+def absmean_gamma(w_bits: np.ndarray) -> np.float32:
+    """gamma = fp32( fp64( sum |W| ) / n ), the sum rounded once.
+
+    math.fsum returns the correctly rounded (round-half-even) fp64 value of
+    the exact sum of its inputs; bf16 magnitudes are exact in fp64.
+    """
+    n = w_bits.size
+    mags = np.abs(bf16_to_f32(w_bits).astype(np.float64)).ravel()
+    total = math.fsum(mags)
+    return np.float32(total / float(n))
+
+
+# --------------------------------------------------------------------------
+# (a3) ternary quantiser and quant-then-mask
+# [summary] 前置知识: W_q = RoundClip(W / gamma, -1, +1); epsilon in the
+# denominator per the plain reading of the operator spec; [summary] 核心方法
+# (iii): W_eff = W_q (.) M_{N:M}; [explainer] "1.58 位元量化的技術原理"
+# (threshold form -1 / 0 / +1 at -gamma/2, +gamma/2).
+# --------------------------------------------------------------------------
+def ternary(w_bits: np.ndarray, gamma: np.float32) -> np.ndarray:
+    """W_q = clip(rint(fp32(w / fp32(gamma + eps))), -1, 1) as int8.
+
+    rint rounds half to even, so |w / den| = 0.5 maps to 0.
+    """
+    w = bf16_to_f32(w_bits)
+    den = np.float32(np.float32(gamma) + EPS)
+    r = np.divide(w, den, dtype=np.float32)
+    return np.clip(np.rint(r), -1.0, 1.0).astype(np.int8)
+
+
+def effective_weight(w_bits: np.ndarray, N: int, M: int):
+    """Algorithm 1 steps (2), (4), (5): returns (W_eff int8, gamma fp32,
+    keep bool).  The mask comes from |W|, not from W_q."""
+    keep = nm_mask(w_bits, N, M)
+    gamma = absmean_gamma(w_bits)
+    wq = ternary(w_bits, gamma)
+    weff = np.where(keep, wq, np.int8(0)).astype(np.int8)
+    return weff, gamma, keep
+
+
+# --------------------------------------------------------------------------
+# (a4) per-token absmax int8 activation quantisation
+# [summary] 前置知识 ("激活值另用 absmax 量化到 8-bit 整数") and Algorithm 1
+# step (3).
+# --------------------------------------------------------------------------
+def act_quant(x_bits: np.ndarray):
+    """Returns (X_q int8 [T, d_in], amax fp32 [T]).
+
+    amax_t = max(max_j |x_tj|, 1e-5); s_t = fp32(127 / amax_t);
+    X_q = clip(rint(fp32(x * s_t)), -128, 127).
+    """
+    x = bf16_to_f32(x_bits)
+    if x.shape[0] == 0:
+        return np.zeros(x.shape, np.int8), np.zeros((0,), np.float32)
+    a = np.abs(x).max(axis=1).astype(np.float32)
+    a = np.maximum(a, ACT_FLOOR)
+    s = np.divide(QMAX, a, dtype=np.float32)
+    xs = np.multiply(x, s[:, None], dtype=np.float32)
+    xq = np.clip(np.rint(xs), -128.0, 127.0).astype(np.int8)
+    return xq, a
+
+
+# --------------------------------------------------------------------------
+# (a5) forward: y = (X_q . W_eff^T) * gamma * amax / 127, int32 accumulation
+# [summary] Algorithm 1 step (6) ("y ~ s * W_eff x~", s absorbs the scales);
+# [summary] 半结构化 N:M 稀疏 (y = (W (.) M) x).
+# --------------------------------------------------------------------------
+def forward_acc(xq: np.ndarray, weff: np.ndarray) -> np.ndarray:
+    """acc[t, o] = sum_j xq[t, j] * W_eff[o, j], exact integers (int32)."""
+    acc = xq.astype(np.int64) @ weff.astype(np.int64).T
+    return acc.astype(np.int32)
+
+
+def forward_out(acc: np.ndarray, gamma: np.float32, amax: np.ndarray) -> np.ndarray:
+    """y = fp32( fp32(acc) * fp32(gamma * fp32(amax / 127)) )."""
+    c = np.divide(amax.astype(np.float32), QMAX, dtype=np.float32)
+    sc = np.multiply(np.float32(gamma), c, dtype=np.float32)
+    return np.multiply(acc.astype(np.float32), sc[:, None], dtype=np.float32)
+
+
+def forward(x_bits: np.ndarray, w_bits: np.ndarray, N: int, M: int):
+    """Whole forward of one Sparse-BitLinear layer.  Returns a dict."""
+    weff, gamma, keep = effective_weight(w_bits, N, M)
+    xq, amax = act_quant(x_bits)
+    acc = forward_acc(xq, weff)
+    y = forward_out(acc, gamma, amax)
+    return dict(weff=weff, gamma=gamma, keep=keep, xq=xq, amax=amax, acc=acc, y=y)
+
+
+# --------------------------------------------------------------------------
+# (a6, a7) Dual-STE backward
+# [summary] Straight-Through Estimator (Q replaced by the identity in the
+# backward; Dual STE extends it to Pi_{N:M}); [summary] 核心方法 (masked
+# weights receive the full gradient); Algorithm 1 step (7); [gist] 2.2.
+# --------------------------------------------------------------------------
+def backward_dx(dy_bits: np.ndarray, weff: np.ndarray, gamma: np.float32) -> np.ndarray:
+    """dX = dY . (gamma * W_eff), fp64 accumulation, fp32 result."""
+    dy = bf16_to_f32(dy_bits).astype(np.float64)
+    return (float(gamma) * (dy @ weff.astype(np.float64))).astype(np.float32)
+
+
+def backward_dw(dy_bits: np.ndarray, x_bits: np.ndarray) -> np.ndarray:
+    """dW = dY^T . X (dense, unmasked), fp64 accumulation, fp32 result."""
+    dy = bf16_to_f32(dy_bits).astype(np.float64)
+    x = bf16_to_f32(x_bits).astype(np.float64)
+    return (dy.T @ x).astype(np.float32)
+
+
+# --------------------------------------------------------------------------
+# (a9) packed inference format: 2-bit ternary codes + N:M index
+# [article] 7.1 推理优化技巧 (pre-compute and cache the sparse format; bit
+# operations for ternary products); [summary] 核心方法 (the deployed ternary
+# weights are N:M-structured).
+#
+# Per weight row, two planes, each padded to a multiple of 16 bytes:
+#   codes plane: for every group of M, the codes of its N slots in ascending
+#     position order, 2 bits each (00 -> 0, 01 -> +1, 11 -> -1), written as
+#     a little-endian bit stream (code i of group g at bit 2*(g*N + i));
+#   index plane: for every group, an M-bit slot mask (bit p = position p is a
+#     slot), little-endian bit stream (group g at bit g*M).
+# Slots are all nonzero positions of the group plus, if there are fewer
+# than N, the lowest-index zero positions.  The buffer holds all code rows
+# first, then all index rows.
+# --------------------------------------------------------------------------
+def _ceil16(n: int) -> int:
+    return (n + 15) // 16 * 16
+
+
+def packed_layout(d_out: int, d_in: int, N: int, M: int):
+    """(codes_row_bytes, index_row_bytes, total_bytes)."""
+    G = d_in // M
+    crow = _ceil16((G * N * 2 + 7) // 8)
+    irow = _ceil16((G * M + 7) // 8)
+    return crow, irow, d_out * (crow + irow)
+
+
+def _put_bits(buf: bytearray, bitpos: int, value: int, nbits: int) -> None:
+    for b in range(nbits):
+        if (value >> b) & 1:
+            buf[(bitpos + b) // 8] |= 1 << ((bitpos + b) % 8)
+
+
+def _get_bits(buf, bitpos: int, nbits: int) -> int:
+    v = 0
+    for b in range(nbits):
+        if (buf[(bitpos + b) // 8] >> ((bitpos + b) % 8)) & 1:
+            v |= 1 << b
+    return v
+
+
+_CODE = {0: 0b00, 1: 0b01, -1: 0b11}
+_VALUE = {0b00: 0, 0b01: 1, 0b11: -1}
+
+
+def pack(weff: np.ndarray, N: int, M: int) -> np.ndarray:
+    """Pack W_eff (int8 in {-1,0,1}, at most N nonzeros per group)."""
+    d_out, d_in = weff.shape
+    crow, irow, total = packed_layout(d_out, d_in, N, M)
+    G = d_in // M
+    out = bytearray(total)
+    for o in range(d_out):
+        codes = bytearray(crow)
+        index = bytearray(irow)
+        for g in range(G):
+            grp = [int(v) for v in weff[o, g * M:(g + 1) * M]]
+            nz = [p for p in range(M) if grp[p] != 0]
+            if len(nz) > N:
+                raise ValueError(f"row {o} group {g}: {len(nz)} nonzeros > N={N}")
+            zeros = [p for p in range(M) if grp[p] == 0]
+            slots = sorted(nz + zeros[: N - len(nz)])
+            _put_bits(index, g * M, sum(1 << p for p in slots), M)
+            for i, p in enumerate(slots):
+                _put_bits(codes, 2 * (g * N + i), _CODE[grp[p]], 2)
+        out[o * crow:(o + 1) * crow] = codes
+        base = d_out * crow
+        out[base + o * irow: base + (o + 1) * irow] = index
+    return np.frombuffer(bytes(out), dtype=np.uint8).copy()
+
+
+def unpack(packed: np.ndarray, d_out: int, d_in: int, N: int, M: int) -> np.ndarray:
+    """Inverse of :func:`pack` (raises on an invalid code or slot count)."""
+    crow, irow, total = packed_layout(d_out, d_in, N, M)
+    assert packed.size == total
+    G = d_in // M
+    buf = packed.tobytes()
+    w = np.zeros((d_out, d_in), dtype=np.int8)
+    base = d_out * crow
+    for o in range(d_out):
+        codes = buf[o * crow:(o + 1) * crow]
+        index = buf[base + o * irow: base + (o + 1) * irow]
+        for g in range(G):
+            m = _get_bits(index, g * M, M)
+            slots = [p for p in range(M) if (m >> p) & 1]
+            if len(slots) != N:
+                raise ValueError(f"row {o} group {g}: {len(slots)} slots != N={N}")
+            for i, p in enumerate(slots):
+                c = _get_bits(codes, 2 * (g * N + i), 2)
+                if c not in _VALUE:
+                    raise ValueError(f"row {o} group {g}: invalid code {c:#b}")
+                w[o, g * M + p] = _VALUE[c]
+    return w
+
+
+# --------------------------------------------------------------------------
+# (a10) decode GEMV on the packed format
+# [summary] 实验结果 / Table 3 (decode on the deployed 6:8 ternary model).
+# --------------------------------------------------------------------------
+def gemv_packed(xq: np.ndarray, amax: np.ndarray, packed: np.ndarray,
+                gamma: np.float32, d_in: int, d_out: int, N: int, M: int) -> np.ndarray:
+    """y = forward_out(X_q . unpack(packed)^T, gamma, amax)."""
+    w = unpack(packed, d_out, d_in, N, M)
+    return forward_out(forward_acc(xq, w), gamma, amax)
