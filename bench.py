@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Sparse-BitLinear training-step benchmark (forward + Dual-STE backward).
+
+One step = the whole hot path over one batch of the Qwen2.5-3B-shaped layer
+set (q/o 2048x2048, k/v 256x2048, gate/up 11008x2048, down 2048x11008),
+32768 tokens (16 x 2048), 6:8:
+
+  for every projection:  sbl_mask_quant   (mask, gamma, ternary, quant-then-mask)
+  for every input:       sbl_act_quant    (attn_in, o_in, mlp_in, down_in)
+  for every projection:  sbl_forward      (int8 tcgen05 product)
+                         sbl_backward     (bf16 tcgen05 dX, then dW)
+
+Inputs are seeded synthetic tensors (synth): trimodal bf16 master weights,
+X ~ N(0, 1) with 0.1% outlier channels x10, dY ~ N(0, 1).  The per-step
+working set (about 11 GB) is far larger than the 126 MB L2, so no L2 flush
+is needed between steps.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
+a bounded sample of the same workload instead.  Under torchrun (N > 1) each
+rank runs an independent batch (weak scaling); there is no collective on the
+data path.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "qwen2.5-3b"
+T_TOKENS = 32768
+N_KEEP, M_GROUP = 6, 8
+METRIC = "Sparse-BitLinear fwd+bwd tokens/s (3B-shape, 6:8)"
+
+NOMINAL_I8_OVER_BF16 = 2.0  # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d.get("bf16_tflops_sustained",
+                    d["bf16_tflops"]), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+# ----------------------------------------------------------------- inputs
+def make_inputs(ls, T, seed, device):
+    """Seeded synthetic tensors for one step, on `device` (CPU pinned or cuda)."""
+    W, X, dY = {}, {}, {}
+    for i, p in enumerate(ls.projections):
+        W[p.name] = synth.trimodal_weight(p.d_out, p.d_in, seed=0, tensor_id=i)  # replicated weights
+    for j, (name, d_in) in enumerate(ls.inputs.items()):
+        X[name] = synth.activations(T, d_in, seed=seed, tensor_id=100 + j, outlier_frac=0.001)
+    for i, p in enumerate(ls.projections):
+        dY[p.name] = synth.grad_output(T, p.d_out, seed=seed, tensor_id=200 + i)
+    if device == "pinned":
+        f = lambda t: t.pin_memory()  # noqa: E731
+    else:
+        f = lambda t: t.to(device)  # noqa: E731
+    return ({k: f(v) for k, v in W.items()}, {k: f(v) for k, v in X.items()},
+            {k: f(v) for k, v in dY.items()})
+
+
+class Step:
+    """Device buffers for one step and the sequence of C-ABI calls."""
+
+    def __init__(self, ls, T, W, X, dY):
+        import semi_structured_sparsity_step_b200 as sbl
+        from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer
+        self.sbl, self.ls, self.T = sbl, ls, T
+        self.W, self.X, self.dY = W, X, dY
+        dev = "cuda"
+        self.layers = {p.name: SparseBitLinearLayer(W[p.name], N_KEEP, M_GROUP) for p in ls.projections}
+        self.Xq = {n: torch.empty(T, d, dtype=torch.int8, device=dev) for n, d in ls.inputs.items()}
+        self.amax = {n: torch.empty(T, dtype=torch.float32, device=dev) for n in ls.inputs}
+        self.Y = {p.name: torch.empty(T, p.d_out, dtype=torch.float32, device=dev) for p in ls.projections}
+        self.dX = {p.name: torch.empty(T, p.d_in, dtype=torch.float32, device=dev) for p in ls.projections}
+        self.dW = {p.name: torch.empty(p.d_out, p.d_in, dtype=torch.float32, device=dev) for p in ls.projections}
+        self.kernels_per_step = 2 * 7 + 4 + 7 + 7 + 7
+
+    def run(self, stream, ev=None):
+        """Enqueue one step.  With `ev` (dict name -> list), record event pairs per call."""
+        sbl, ls, T = self.sbl, self.ls, self.T
+
+        def timed(name, fn):
+            if ev is None:
+                fn()
+                return
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ev.setdefault(name, []).append((a, b))
+
+        for p in ls.projections:
+            timed("mask_quant", lambda p=p: self.layers[p.name].weight_step(stream))
+        for n, d in ls.inputs.items():
+            timed("act_quant", lambda n=n, d=d: sbl.sbl_act_quant(self.X[n], T, d, self.Xq[n], self.amax[n],
+                                                                  stream))
+        for p in ls.projections:
+            L = self.layers[p.name]
+            timed("forward_i8", lambda p=p, L=L: L.forward(self.Xq[p.input_name], self.amax[p.input_name],
+                                                           self.Y[p.name], stream=stream))
+        for p in ls.projections:
+            L = self.layers[p.name]
+            timed("backward_dx_bf16", lambda p=p, L=L: L.backward(self.dY[p.name], self.X[p.input_name],
+                                                                  self.dX[p.name], None, stream=stream))
+            timed("backward_dw_bf16", lambda p=p, L=L: L.backward(self.dY[p.name], self.X[p.input_name],
+                                                                  None, self.dW[p.name], stream=stream))
+
+
+def algorithmic_work(ls, T):
+    P = ls.params
+    fwd_ops = 2.0 * T * P          # dense-equivalent int8 ops
+    dx_flops = 2.0 * T * P
+    dw_flops = 2.0 * T * P
+    return fwd_ops, dx_flops, dw_flops
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- CPU oracle timing
+def oracle_sample(ls, T_full, tokens=16, seed=0):
+    """Time the oracle as it stands on a bounded sample of the workload and
+    extrapolate to one full step: the weight side of the q projection scaled
+    by parameter count, the token side of all projections on `tokens` tokens
+    scaled to T_full tokens."""
+    import oracle
+    q = ls.projections[0]
+    wq = synth.bits(synth.trimodal_weight(q.d_out, q.d_in, seed=0, tensor_id=0))
+    t0 = time.perf_counter()
+    oracle.effective_weight(wq, N_KEEP, M_GROUP)
+    t_w = time.perf_counter() - t0
+    weight_side = t_w * ls.params / (q.d_out * q.d_in)
+    xs = {n: synth.bits(synth.activations(tokens, d, seed=seed, tensor_id=100 + j, outlier_frac=0.001))
+          for j, (n, d) in enumerate(ls.inputs.items())}
+    t_tok = 0.0
+    weffs = {}
+    for i, p in enumerate(ls.projections):
+        w = synth.bits(synth.trimodal_weight(p.d_out, p.d_in, seed=0, tensor_id=i))
+        weffs[p.name] = oracle.effective_weight(w, N_KEEP, M_GROUP)
+    for n in ls.inputs:
+        t0 = time.perf_counter()
+        oracle.act_quant(xs[n])
+        t_tok += time.perf_counter() - t0
+    for i, p in enumerate(ls.projections):
+        weff, gamma, _ = weffs[p.name]
+        dy = synth.bits(synth.grad_output(tokens, p.d_out, seed=seed, tensor_id=200 + i))
+        xq, amax = oracle.act_quant(xs[p.input_name])
+        t0 = time.perf_counter()
+        oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax)
+        oracle.backward_dx(dy, weff, gamma)
+        oracle.backward_dw(dy, xs[p.input_name])
+        t_tok += time.perf_counter() - t0
+    token_side = t_tok * T_full / tokens
+    step_s = weight_side + token_side
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([1] + [d.get("num_threads", 1) for d in threadpool_info()])
+    except Exception:  # pragma: no cover
+        cores = 1
+    sample = (f"oracle weight side on q ({q.d_out}x{q.d_in}) scaled x{ls.params / (q.d_out * q.d_in):.2f} by "
+              f"parameter count + token side of all 7 projections on {tokens} tokens scaled x{T_full // tokens}; "
+              f"extrapolated")
+    return step_s, cores, sample, t_w + t_tok
+
+
+# ----------------------------------------------------------------- traffic (ncu)
+def _kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "sbl_device.cuh"):
+        h.update(open(os.path.join(ROOT, "semi_structured_sparsity_step_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_key):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != _kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["sbl", "reference"], default="sbl")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    ls = synth.layer_set(WORKLOAD)
+    T = T_TOKENS
+    config = {"workload": f"{WORKLOAD} layer set (q/o 2048x2048, k/v 256x2048, gate/up 11008x2048, "
+                          f"down 2048x11008), {T} tokens (16 x 2048), N:M {N_KEEP}:{M_GROUP}, trimodal bf16 "
+                          f"master W, X ~ N(0,1) with 0.1% outlier channels x10, dY ~ N(0,1)",
+              "tokens_per_step": T, "params": ls.params, "nm": f"{N_KEEP}:{M_GROUP}",
+              "l2": "inputs larger than L2 (~11 GB per step), no flush", "parallelism": f"dp{args.gpus} replicas"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        step_s, cores, sample, spent = oracle_sample(ls, T)
+        v = T / step_s
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8/bf16 (oracle: fp32/fp64/int64 on CPU)",
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
+                             "cpu_seconds_spent": spent},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    import semi_structured_sparsity_step_b200 as sbl
+    sbl.load()
+
+    stream = torch.cuda.Stream()
+    Wp, Xp, dYp = make_inputs(ls, T, seed=rank, device="pinned")
+    with torch.cuda.stream(stream):
+        W = {k: v.to("cuda", non_blocking=True) for k, v in Wp.items()}
+        X = {k: v.to("cuda", non_blocking=True) for k, v in Xp.items()}
+        dY = {k: v.to("cuda", non_blocking=True) for k, v in dYp.items()}
+        step = Step(ls, T, W, X, dY)
+    stream.synchronize()
+
+    for _ in range(args.warmup):
+        step.run(stream)
+    sbl.sbl_check(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- device-timed steps (inputs resident in HBM)
+    ev = {}
+    barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            step.run(stream, ev)
+        end.record(stream)
+        stream.synchronize()
+    barrier()
+    sbl.sbl_check(stream)
+    elapsed_ms = start.elapsed_time(end)
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = t.item()
+    ms_per_step = elapsed_ms / args.steps
+    value = world * T / (ms_per_step / 1e3)
+
+    per_call = {k: sum(a.elapsed_time(b) for a, b in v) / args.steps for k, v in ev.items()}
+    launches = {k: len(v) // args.steps for k, v in ev.items()}
+
+    # ---- end to end through host buffers (pinned), copies inside the timed region
+    h2d = sum(t.numel() * t.element_size() for d in (Wp, Xp, dYp) for t in d.values())
+    outs = [*step.Y.values(), *step.dX.values(), *step.dW.values()]
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.e2e_steps):
+            for src, dst in ((Wp, W), (Xp, X), (dYp, dY)):
+                for k in src:
+                    dst[k].copy_(src[k], non_blocking=True)
+            step.run(stream)
+            for h, d in zip(host_out, outs):
+                h.copy_(d, non_blocking=True)
+    e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    e2e_value = world * T / (e2e_ms / 1e3)
+
+    # ---- roofline of the dominant call family and of the whole step
+    pk = peaks()
+    fwd_ops, dx_flops, dw_flops = algorithmic_work(ls, T)
+    work = {"forward_i8": (fwd_ops, pk["bf16_sust"] * NOMINAL_I8_OVER_BF16),
+            "backward_dx_bf16": (dx_flops, pk["bf16_sust"]),
+            "backward_dw_bf16": (dw_flops, pk["bf16_sust"])}
+    dom = max(work, key=lambda k: per_call.get(k, 0.0))
+    flops, peak_tf = work[dom]
+    n_launch = launches[dom]
+    achieved_tf = (flops / n_launch) / ((per_call[dom] / n_launch) / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved_tf / peak_tf, "traffic": traffic_for(dom),
+                "peak_source": f"{pk['src']} bf16 sustained" + (" x2 nominal int8/bf16" if dom == "forward_i8"
+                                                                 else ""),
+                "per_launch_work": flops / n_launch, "launches_per_step": n_launch,
+                "note": "achieved = dense-equivalent algorithmic ops of the 7 projections / summed CUDA-event "
+                        "time of those launches in the timed region"}
+    t_roof = fwd_ops / (pk["bf16_sust"] * NOMINAL_I8_OVER_BF16 * 1e12) + (dx_flops + dw_flops) / (
+        pk["bf16_sust"] * 1e12)
+    step_roofline = {"roofline_ms": t_roof * 1e3, "measured_ms": ms_per_step, "frac": t_roof * 1e3 / ms_per_step,
+                     "basis": "dense-equivalent int8 fwd + bf16 dX, dW on measured sustained peaks"}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        step_s, cores, sample, spent = oracle_sample(ls, T)
+        cpu = {"value": T / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
+               "cpu_seconds_spent": spent}
+
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "i8 fwd / bf16 bwd (fp32 accumulate)", "data": "synthetic",
+            "config": config, "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": step.kernels_per_step * args.steps,
+            "per_call_ms_per_step": per_call, "clocks": clk.summary(),
+        }))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,179 @@
+/*
+ * sbl.h -- C ABI of the Sparse-BitLinear operator for NVIDIA B200 (sm_100a).
+ *
+ * Sparse-BitLinear is the layer of Sparse-BitNet: per step it recomputes an
+ * N:M magnitude mask on the bf16 master weight W, quantises W to ternary
+ * with an absmean scale, masks the ternary weight, quantises activations
+ * per token to int8, multiplies on int8 tensor cores, and back-propagates
+ * with a "Dual" straight-through estimator that gives masked weights their
+ * full gradient.
+ *
+ * Pages cited below (by title and section):
+ *   [summary]   "Sparse-BitNet：1.58-bit 大模型天然兼容半结构化稀疏", the
+ *               structured summary of arXiv 2603.05168: 前置知识 (1.58-bit
+ *               BitNet 量化; 半结构化 N:M 稀疏; STE), 核心方法,
+ *               方法步骤详情 (Algorithm 1), 实验结果 (Table 3).
+ *   [explainer] "什麼是 Sparse-BitNet？核心概念一次搞懂": 1.58 位元量化的技術原理;
+ *               N:M 半結構化稀疏性的運作機制.
+ *   [article]   "突破性发现：极低位量化与稀疏化的完美协同": 7.1 推理优化技巧.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers (CUDA global memory) owned by
+ *     the caller; the library never frees or retains them.  The library
+ *     allocates no device memory except fixed-size static state created on
+ *     first use (tensor-map encoder entry point, attribute settings).
+ *   - Matrices are row-major with the last index contiguous.  "bf16" means
+ *     IEEE bfloat16 bit patterns (uint16 per element).
+ *   - Every pointer must be 16-byte aligned.  d_in must be a multiple of 16
+ *     and of M; d_out must be a multiple of 8.  T (tokens) may be any value
+ *     >= 0; T = 0 is a no-op.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work on `stream` and returns; it
+ *     never synchronises.
+ *   - Return value: SBL_OK, or an error code.  Argument errors are detected on
+ *     the host before anything is launched and leave all outputs untouched.
+ *     Launch failures return SBL_ERR_CUDA.  Errors found by a kernel while it
+ *     runs (a bounded wait that expired, a pack input with more than N
+ *     nonzeros in a group) are latched in a device word and returned by the
+ *     next sbl_check() on that device.
+ *   - No call throws or aborts across the ABI.
+ */
+#ifndef SBL_H_
+#define SBL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SBL_OK = 0,
+  SBL_ERR_INVALID_ARG = 1, /* null pointer, N/M out of range, bad flag       */
+  SBL_ERR_SHAPE = 2,       /* d_in % 16, d_in % M, d_out % 8, negative sizes */
+  SBL_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                */
+  SBL_ERR_UNSUPPORTED = 4, /* device is not sm_100, or an unsupported N:M     */
+  SBL_ERR_WORKSPACE = 5,   /* workspace (or packed buffer) too small          */
+  SBL_ERR_TIMEOUT = 6,     /* a kernel's bounded wait expired (latched)       */
+  SBL_ERR_CUDA = 7,        /* a CUDA runtime call failed                      */
+  SBL_ERR_DEVICE_CHECK = 8 /* a kernel rejected its input data (latched)      */
+} sbl_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sbl_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int sbl_version(void);
+
+/* Synchronise `stream`, then return (and clear) the first error latched by a
+ * kernel of this library on the current device since the previous check;
+ * SBL_OK if none.  Also reports a pending CUDA error as SBL_ERR_CUDA. */
+sbl_status sbl_check(void* stream);
+
+/* ------------------------------------------------------------------------
+ * Weight side: mask, absmean scale, ternary quantiser, quant-then-mask.
+ * [summary] 前置知识 / 1.58-bit BitNet 量化: gamma = ||W||_1/(d_out*d_in),
+ *   W_q = RoundClip(W/(gamma+eps), -1, +1), eps = 1e-5, round half to even;
+ * [summary] 半结构化 N:M 稀疏 and 核心方法 (i)-(iii), Algorithm 1 steps
+ *   (2), (4), (5): keep the top-N of |W| among each M consecutive weights
+ *   along d_in (ties -> lowest index), W_eff = W_q (.) mask.
+ *
+ *   W          [d_out, d_in] bf16, read only.
+ *   N, M       M in {4, 8}, 1 <= N <= M.
+ *   W_eff      [d_out, d_in] int8 out, values in {-1, 0, +1}.
+ *   W_eff_bf16 optional (NULL): [d_out, d_in] bf16 out, the same values as
+ *              exact bf16 (the operand of the backward dX product).
+ *   mask_bits  optional (NULL): [d_out, d_in/8] uint8 out; bit p of byte b of
+ *              a row is the keep flag of weight 8*b + p of that row.
+ *   gamma      1 float out (device): the absmean scale.  It is the exact
+ *              sum of |W| rounded once to fp64, divided by d_out*d_in in
+ *              fp64, rounded to fp32.
+ *   workspace  device scratch of at least sbl_mask_quant_workspace_bytes()
+ *              bytes, 256-byte aligned; contents on entry are ignored.
+ *              Calls that share a workspace must be ordered on one stream.
+ * ---------------------------------------------------------------------- */
+size_t sbl_mask_quant_workspace_bytes(int d_out, int d_in);
+sbl_status sbl_mask_quant(const void* W, int d_out, int d_in, int N, int M,
+                          int8_t* W_eff, void* W_eff_bf16, uint8_t* mask_bits,
+                          float* gamma, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* ------------------------------------------------------------------------
+ * Per-token absmax int8 activation quantiser.
+ * [summary] 前置知识 (activations absmax-quantised to 8-bit integers) and
+ * Algorithm 1 step (3).
+ *   X     [T, d_in] bf16 in.
+ *   Xq    [T, d_in] int8 out: clip(rint(fp32(x * fp32(127 / amax_t))), -128, 127).
+ *   amax  [T] float out: amax_t = max(max_j |x_tj|, 1e-5).
+ * ---------------------------------------------------------------------- */
+sbl_status sbl_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* amax,
+                         void* stream);
+
+/* ------------------------------------------------------------------------
+ * Forward product on int8 tensor cores (tcgen05, int32 accumulation).
+ * [summary] Algorithm 1 step (6): y = s * W_eff x~, with s absorbing the
+ * quantisation scales: y[t,o] = fp32(fp32(acc) * fp32(gamma * fp32(amax_t/127))),
+ * acc[t,o] = sum_j Xq[t,j] * W_eff[o,j] (exact int32).
+ *   Xq     [T, d_in] int8, amax [T] float (from sbl_act_quant).
+ *   W_eff  [d_out, d_in] int8 (from sbl_mask_quant), gamma 1 float (device).
+ *   Y      [T, d_out] float out.
+ *   acc    optional (NULL): [T, d_out] int32 out, the raw accumulators.
+ * ---------------------------------------------------------------------- */
+sbl_status sbl_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff,
+                       const float* gamma, int T, int d_in, int d_out, float* Y,
+                       int32_t* acc, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dual-STE backward on bf16 tensor cores (tcgen05, fp32 accumulation).
+ * [summary] 前置知识 / STE and 核心方法 (masked weights receive the full
+ * gradient), Algorithm 1 step (7):
+ *   dX = gamma * (dY . W_eff)          [T, d_in]
+ *   dW = dY^T . X  (dense, unmasked)   [d_out, d_in]
+ *   dY          [T, d_out] bf16;  X [T, d_in] bf16 (the layer input);
+ *   W_eff_bf16  [d_out, d_in] bf16 (from sbl_mask_quant); gamma 1 float.
+ *   dX          optional (NULL skips it): [T, d_in] float out.
+ *   dW          optional (NULL skips it): [d_out, d_in] float out;
+ *               accumulate_dW != 0 adds into the existing contents (gradient
+ *               accumulation), 0 overwrites.
+ *   workspace   device scratch of sbl_backward_workspace_bytes() bytes (may
+ *               be NULL when that is 0).
+ * ---------------------------------------------------------------------- */
+size_t sbl_backward_workspace_bytes(int T, int d_in, int d_out);
+sbl_status sbl_backward(const void* dY, const void* X, const void* W_eff_bf16,
+                        const float* gamma, int T, int d_in, int d_out, float* dX,
+                        float* dW, int accumulate_dW, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Packed inference format: 2-bit ternary codes + N:M slot index.
+ * [article] 7.1 (pre-compute and cache the sparse format for inference);
+ * [summary] 核心方法 (masking after quantisation makes the deployed ternary
+ * weights N:M-structured).
+ * Layout, per weight row, two planes each padded to a multiple of 16 bytes:
+ *   codes plane: for every group of M, the N slot codes in ascending position
+ *     order, 2 bits each (00 = 0, 01 = +1, 11 = -1), as a little-endian bit
+ *     stream (code i of group g at bit 2*(g*N + i));
+ *   index plane: the M-bit slot mask of every group (bit p = position p is a
+ *     slot), little-endian bit stream (group g at bit g*M).
+ * Slots are the group's nonzero positions plus, if fewer than N, its lowest
+ * zero positions.  Buffer = d_out code rows, then d_out index rows.
+ * A group with more than N nonzeros latches SBL_ERR_DEVICE_CHECK.
+ * ---------------------------------------------------------------------- */
+size_t sbl_packed_bytes(int d_out, int d_in, int N, int M);
+sbl_status sbl_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M,
+                    uint8_t* packed, size_t packed_bytes, void* stream);
+
+/* Decode GEMV on the packed format, batch 1..16 tokens.
+ * [summary] 实验结果 / Table 3 (decode on the 6:8 ternary model).
+ *   Xq [batch, d_in] int8, amax [batch] float, gamma 1 float (device),
+ *   Y  [batch, d_out] float out, same formula as sbl_forward. */
+sbl_status sbl_gemv_packed(const int8_t* Xq, const float* amax, int batch,
+                           const uint8_t* packed, const float* gamma, int d_in,
+                           int d_out, int N, int M, float* Y, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBL_H_ */

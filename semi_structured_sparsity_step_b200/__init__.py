@@ -1,0 +1,17 @@
+"""B200-native Sparse-BitLinear: CUDA kernels for sm_100a behind a C ABI.
+
+The library (``libsbl.so``, built by ``python -m
+semi_structured_sparsity_step_b200.build``) exports the entry points declared
+in ``include/sbl.h``; this package re-exports their ctypes binding under the
+same names, plus :mod:`.layer`, a small helper that owns the device buffers of
+one Sparse-BitLinear layer and runs its training step through the C ABI.
+"""
+from ._binding import (SblError, load, sbl_act_quant, sbl_backward, sbl_backward_workspace_bytes,  # noqa: F401
+                       sbl_check, sbl_forward, sbl_gemv_packed, sbl_mask_quant, sbl_mask_quant_workspace_bytes,
+                       sbl_pack, sbl_packed_bytes, sbl_status_string, sbl_version)
+
+__all__ = [
+    "SblError", "load", "sbl_act_quant", "sbl_backward", "sbl_backward_workspace_bytes", "sbl_check",
+    "sbl_forward", "sbl_gemv_packed", "sbl_mask_quant", "sbl_mask_quant_workspace_bytes", "sbl_pack",
+    "sbl_packed_bytes", "sbl_status_string", "sbl_version",
+]

@@ -1,0 +1,143 @@
+"""ctypes binding of libsbl.so (the C ABI in include/sbl.h).
+
+Argument marshalling only: each function takes torch tensors (or raw device
+pointers as ints), passes their device pointers, sizes and the current CUDA
+stream to the C entry point of the same name, and raises SblError on a
+non-OK status.  Every computation runs in the library's CUDA kernels; there
+is no fallback path.  Output tensors are allocated by the caller.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libsbl.so")
+
+_c_int = ctypes.c_int
+_c_size = ctypes.c_size_t
+_vp = ctypes.c_void_p
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "sbl_status_string": (ctypes.c_char_p, [_c_int]),
+    "sbl_version": (_c_int, []),
+    "sbl_check": (_c_int, [_vp]),
+    "sbl_mask_quant_workspace_bytes": (_c_size, [_c_int, _c_int]),
+    "sbl_mask_quant": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
+    "sbl_act_quant": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp]),
+    "sbl_forward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
+    "sbl_backward_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
+    "sbl_backward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp, _c_size, _vp]),
+    "sbl_packed_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "sbl_pack": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
+    "sbl_gemv_packed": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
+}
+
+STATUS = {
+    0: "SBL_OK", 1: "SBL_ERR_INVALID_ARG", 2: "SBL_ERR_SHAPE", 3: "SBL_ERR_ALIGN",
+    4: "SBL_ERR_UNSUPPORTED", 5: "SBL_ERR_WORKSPACE", 6: "SBL_ERR_TIMEOUT", 7: "SBL_ERR_CUDA",
+    8: "SBL_ERR_DEVICE_CHECK",
+}
+
+
+class SblError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libsbl.so once; raises if it was not built (no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(
+                f"{path} is missing: build it with `python -m semi_structured_sparsity_step_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _call(name, *args):
+    st = getattr(load(), name)(*args)
+    if st != 0:
+        raise SblError(name, st)
+
+
+def sbl_status_string(status: int) -> str:
+    return load().sbl_status_string(status).decode()
+
+
+def sbl_version() -> int:
+    return load().sbl_version()
+
+
+def sbl_check(stream=None) -> None:
+    _call("sbl_check", _stream(stream))
+
+
+def sbl_mask_quant_workspace_bytes(d_out: int, d_in: int) -> int:
+    return load().sbl_mask_quant_workspace_bytes(d_out, d_in)
+
+
+def sbl_mask_quant(W, d_out, d_in, N, M, W_eff, W_eff_bf16, mask_bits, gamma, workspace, workspace_bytes,
+                   stream=None) -> None:
+    _call("sbl_mask_quant", _ptr(W), d_out, d_in, N, M, _ptr(W_eff), _ptr(W_eff_bf16), _ptr(mask_bits),
+          _ptr(gamma), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def sbl_act_quant(X, T, d_in, Xq, amax, stream=None) -> None:
+    _call("sbl_act_quant", _ptr(X), T, d_in, _ptr(Xq), _ptr(amax), _stream(stream))
+
+
+def sbl_forward(Xq, amax, W_eff, gamma, T, d_in, d_out, Y, acc=None, stream=None) -> None:
+    _call("sbl_forward", _ptr(Xq), _ptr(amax), _ptr(W_eff), _ptr(gamma), T, d_in, d_out, _ptr(Y), _ptr(acc),
+          _stream(stream))
+
+
+def sbl_backward_workspace_bytes(T, d_in, d_out) -> int:
+    return load().sbl_backward_workspace_bytes(T, d_in, d_out)
+
+
+def sbl_backward(dY, X, W_eff_bf16, gamma, T, d_in, d_out, dX, dW, accumulate_dW=0, workspace=None,
+                 workspace_bytes=0, stream=None) -> None:
+    _call("sbl_backward", _ptr(dY), _ptr(X), _ptr(W_eff_bf16), _ptr(gamma), T, d_in, d_out, _ptr(dX), _ptr(dW),
+          int(accumulate_dW), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def sbl_packed_bytes(d_out, d_in, N, M) -> int:
+    return load().sbl_packed_bytes(d_out, d_in, N, M)
+
+
+def sbl_pack(W_eff, d_out, d_in, N, M, packed, packed_bytes, stream=None) -> None:
+    _call("sbl_pack", _ptr(W_eff), d_out, d_in, N, M, _ptr(packed), packed_bytes, _stream(stream))
+
+
+def sbl_gemv_packed(Xq, amax, batch, packed, gamma, d_in, d_out, N, M, Y, stream=None) -> None:
+    _call("sbl_gemv_packed", _ptr(Xq), _ptr(amax), batch, _ptr(packed), _ptr(gamma), d_in, d_out, N, M, _ptr(Y),
+          _stream(stream))

@@ -1,0 +1,130 @@
+// act_quant.cu -- (a4) per-token absmax int8 activation quantiser on sm_100a.
+//
+// Sparse-BitNet summary ("Sparse-BitNet：1.58-bit 大模型天然兼容半结构化稀疏"),
+// 前置知识 (activations absmax-quantised to 8-bit integers) and Algorithm 1
+// step (3):
+//   amax_t = max(max_j |x_tj|, 1e-5),  s_t = fp32(127 / amax_t),
+//   Xq[t, j] = clip(rint(fp32(x_tj * s_t)), -128, 127).
+//
+// HBM bound: each row is read once with 128-bit loads into registers (up to
+// 8 x 16 bytes per thread), reduced (integer max over the 15-bit bf16
+// magnitudes, which orders like the values), then quantised from registers.
+// TPR threads share a row: 32 for d_in <= 2048, up to 256 for d_in <= 16384;
+// longer rows re-read the uncached tail from L2.
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "sbl_device.cuh"
+#include "sbl_internal.h"
+
+namespace sbl {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kVpt = 8;
+
+__device__ __forceinline__ uint32_t max_mag8(const uint4& v) {
+  uint32_t m = 0;
+  const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    m = max(m, w4[k] & 0x7FFFu);
+    m = max(m, (w4[k] >> 16) & 0x7FFFu);
+  }
+  return m;
+}
+
+__device__ __forceinline__ uint32_t quant4(uint32_t lo_pair, uint32_t hi_pair, float s) {
+  const uint32_t h[4] = {lo_pair & 0xFFFFu, lo_pair >> 16, hi_pair & 0xFFFFu, hi_pair >> 16};
+  uint32_t out = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float x = __uint_as_float(h[k] << 16);
+    float r = rintf(__fmul_rn(x, s));
+    r = fminf(fmaxf(r, -128.0f), 127.0f);
+    out |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu) << (8 * k);
+  }
+  return out;
+}
+
+template <int TPR>
+__global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint4* __restrict__ X, int T, int nv,
+                                                             uint2* __restrict__ Xq, float* __restrict__ amax) {
+  constexpr int RPB = kThreads / TPR;      // rows per block
+  constexpr int WPR = TPR / 32;            // warps per row
+  __shared__ uint32_t s_max[kThreads / 32];
+  const int rib = threadIdx.x / TPR;
+  const int tr = threadIdx.x % TPR;
+  const int warp = threadIdx.x >> 5;
+
+  for (long long base = static_cast<long long>(blockIdx.x) * RPB; base < T;
+       base += static_cast<long long>(gridDim.x) * RPB) {
+    const long long row = base + rib;
+    const bool active = row < T;
+    const uint4* xr = X + row * static_cast<long long>(nv);
+    uint4 v[kVpt];
+    uint32_t mx = 0;
+#pragma unroll
+    for (int k = 0; k < kVpt; ++k) {
+      const int idx = tr + k * TPR;
+      if (active && idx < nv) {
+        v[k] = __ldg(xr + idx);
+        mx = max(mx, max_mag8(v[k]));
+      } else {
+        v[k] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    if (active) {
+      for (int idx = tr + kVpt * TPR; idx < nv; idx += TPR) mx = max(mx, max_mag8(__ldg(xr + idx)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if constexpr (WPR > 1) {
+      if ((threadIdx.x & 31) == 0) s_max[warp] = mx;
+      __syncthreads();
+      mx = 0;
+#pragma unroll
+      for (int w = 0; w < WPR; ++w) mx = max(mx, s_max[rib * WPR + w]);
+      __syncthreads();
+    }
+    if (!active) continue;
+    const float a = fmaxf(__uint_as_float(mx << 16), 1e-5f);
+    const float s = __fdiv_rn(127.0f, a);
+    uint2* qr = Xq + row * static_cast<long long>(nv);
+#pragma unroll
+    for (int k = 0; k < kVpt; ++k) {
+      const int idx = tr + k * TPR;
+      if (idx < nv) qr[idx] = make_uint2(quant4(v[k].x, v[k].y, s), quant4(v[k].z, v[k].w, s));
+    }
+    for (int idx = tr + kVpt * TPR; idx < nv; idx += TPR) {
+      const uint4 u = __ldg(xr + idx);
+      qr[idx] = make_uint2(quant4(u.x, u.y, s), quant4(u.z, u.w, s));
+    }
+    if (tr == 0) amax[row] = a;
+  }
+}
+
+template <int TPR>
+cudaError_t launch_tpr(const void* X, int T, int nv, int8_t* Xq, float* amax, cudaStream_t stream, int num_sms) {
+  constexpr int RPB = kThreads / TPR;
+  long long blocks = (static_cast<long long>(T) + RPB - 1) / RPB;
+  const long long cap = static_cast<long long>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  act_quant_kernel<TPR><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+      static_cast<const uint4*>(X), T, nv, reinterpret_cast<uint2*>(Xq), amax);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* amax, cudaStream_t stream,
+                             int num_sms) {
+  if (T == 0) return cudaSuccess;
+  const int nv = d_in / 8;
+  if (nv <= 32 * kVpt) return launch_tpr<32>(X, T, nv, Xq, amax, stream, num_sms);
+  if (nv <= 64 * kVpt) return launch_tpr<64>(X, T, nv, Xq, amax, stream, num_sms);
+  if (nv <= 128 * kVpt) return launch_tpr<128>(X, T, nv, Xq, amax, stream, num_sms);
+  return launch_tpr<256>(X, T, nv, Xq, amax, stream, num_sms);
+}
+
+}  // namespace sbl

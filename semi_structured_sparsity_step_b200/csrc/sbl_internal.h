@@ -1,0 +1,47 @@
+// sbl_internal.h -- host-side declarations shared by the library's .cu files
+// (launchers called by the C ABI in sbl_api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace sbl {
+
+// ---- mask / gamma / ternary (mask_quant.cu)
+constexpr int kGammaMaxBlocks = 592;  // 4 blocks of 256 threads per SM on 148 SMs
+constexpr int kGammaLimbs = 10;       // 320-bit exact sum of |W| in units of 2^-133
+
+struct GammaWorkspace {
+  unsigned long long bucket[256];  // sum of 8-bit significands per biased exponent
+  unsigned int ticket;             // blocks finished
+  unsigned int pad[63];
+  unsigned long long block_window[kGammaMaxBlocks];  // per-block window sums
+};
+
+size_t mask_quant_workspace_bytes();
+cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, int8_t* W_eff, void* W_eff_bf16,
+                              uint8_t* mask_bits, float* gamma, void* workspace, cudaStream_t stream, int num_sms);
+
+// ---- activation quantiser (act_quant.cu)
+cudaError_t launch_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* amax, cudaStream_t stream,
+                             int num_sms);
+
+// ---- tensor-core GEMMs (gemm_tc.cu)
+cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
+                           int d_in, int d_out, float* Y, int32_t* acc, cudaStream_t stream, int num_sms,
+                           uint32_t* err);
+cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf16, const float* gamma, int T,
+                            int d_in, int d_out, float* dX, float* dW, int accumulate_dW, cudaStream_t stream,
+                            int num_sms, uint32_t* err);
+
+// ---- packed format (pack_gemv.cu)
+size_t packed_codes_row_bytes(int d_in, int N, int M);
+size_t packed_index_row_bytes(int d_in, int M);
+cudaError_t launch_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M, uint8_t* packed,
+                        cudaStream_t stream, uint32_t* err);
+cudaError_t launch_gemv_packed(const int8_t* Xq, const float* amax, int batch, const uint8_t* packed,
+                               const float* gamma, int d_in, int d_out, int N, int M, float* Y,
+                               cudaStream_t stream, int num_sms);
+
+}  // namespace sbl

@@ -1,0 +1,226 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bit-exact: keep masks, ternary codes (int8 and bf16 copies), gamma, int8
+activations, amax, int32 accumulators, packed bytes.  Float outputs: the
+forward output within a relative 1e-3 (it is computed with the same fp32
+operation order, so it is normally bit-equal); dX and dW (bf16 tensor-core
+products with fp32 accumulation against an fp64 oracle) within
+max|gpu - ref| <= 2e-2 * max|ref| per tensor.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+REL_Y = 1e-3
+REL_BWD = 2e-2
+
+
+def _dev(t):
+    return t.to("cuda")
+
+
+def _unpack_mask(bits: np.ndarray) -> np.ndarray:
+    return np.unpackbits(bits, axis=1, bitorder="little").astype(bool)
+
+
+def _check_bwd(gpu: np.ndarray, ref: np.ndarray, what: str):
+    err = np.abs(gpu.astype(np.float64) - ref.astype(np.float64)).max()
+    scale = np.abs(ref).max()
+    assert err <= REL_BWD * scale, f"{what}: max err {err} vs {REL_BWD} * {scale}"
+
+
+def _check_y(gpu: np.ndarray, ref: np.ndarray):
+    np.testing.assert_allclose(gpu, ref, rtol=REL_Y, atol=REL_Y * np.abs(ref).max() * 1e-3)
+
+
+class Layer:
+    """Runs the whole path for one layer on the GPU and keeps host copies."""
+
+    def __init__(self, lib, w, x, dy, N, M, accumulate=None):
+        from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer, act_quant
+        d_out, d_in = w.shape
+        T = x.shape[0]
+        self.L = SparseBitLinearLayer(_dev(w), N, M, keep_mask=True)
+        self.L.weight_step()
+        X = _dev(x)
+        self.Xq = torch.empty(T, d_in, dtype=torch.int8, device="cuda")
+        self.amax = torch.empty(max(T, 1), dtype=torch.float32, device="cuda")
+        act_quant(X, self.Xq, self.amax)
+        self.Y = torch.empty(T, d_out, dtype=torch.float32, device="cuda")
+        self.acc = torch.empty(T, d_out, dtype=torch.int32, device="cuda")
+        self.L.forward(self.Xq, self.amax, self.Y, acc=self.acc)
+        dY = _dev(dy)
+        self.dX = torch.empty(T, d_in, dtype=torch.float32, device="cuda")
+        self.dW = torch.empty(d_out, d_in, dtype=torch.float32, device="cuda") if accumulate is None \
+            else _dev(accumulate.clone())
+        self.L.backward(dY, X, self.dX, self.dW, accumulate_dW=accumulate is not None)
+        lib.sbl_check()
+        torch.cuda.synchronize()
+
+
+def _full_parity(lib, w, x, dy, N, M):
+    g = Layer(lib, w, x, dy, N, M)
+    wb, xb, dyb = synth.bits(w), synth.bits(x), synth.bits(dy)
+    ref = oracle.forward(xb, wb, N, M)
+    assert np.array_equal(_unpack_mask(g.L.mask_bits.cpu().numpy()), ref["keep"])
+    assert g.L.gamma.item() == float(ref["gamma"])
+    assert np.array_equal(g.L.W_eff.cpu().numpy(), ref["weff"])
+    assert np.array_equal(oracle.bf16_to_f32(synth.bits(g.L.W_eff_bf16.cpu())), ref["weff"].astype(np.float32))
+    assert np.array_equal(g.Xq.cpu().numpy(), ref["xq"])
+    assert np.array_equal(g.amax.cpu().numpy()[: x.shape[0]], ref["amax"])
+    assert np.array_equal(g.acc.cpu().numpy(), ref["acc"])
+    _check_y(g.Y.cpu().numpy(), ref["y"])
+    _check_bwd(g.dX.cpu().numpy(), oracle.backward_dx(dyb, ref["weff"], ref["gamma"]), "dX")
+    _check_bwd(g.dW.cpu().numpy(), oracle.backward_dw(dyb, xb), "dW")
+    return g, ref
+
+
+def test_library_loads_on_gpu(lib):
+    assert lib.sbl_version() >= 100
+    lib.sbl_check()
+
+
+def test_single_layer_256_6of8_full_parity(lib):
+    """One 256 x 256 layer, 64 tokens, 6:8, W ~ N(0, 0.02), X, dY ~ N(0, 1)."""
+    w = synth.normal_weight(256, 256, seed=0, tensor_id=0)
+    x = synth.activations(64, 256, seed=0, tensor_id=100)
+    dy = synth.grad_output(64, 256, seed=0, tensor_id=200)
+    g, ref = _full_parity(lib, w, x, dy, 6, 8)
+    assert np.array_equal(g.Y.cpu().numpy(), ref["y"])  # same fp32 op order: bit-equal
+
+
+@pytest.mark.parametrize("T,d_out,d_in,N,M", [
+    (1, 8, 16, 6, 8), (7, 136, 48, 2, 4), (129, 264, 272, 6, 8), (200, 392, 400, 4, 8),
+    (130, 256, 1040, 3, 4), (333, 520, 144, 8, 8), (64, 8, 2064, 1, 8),
+])
+def test_ragged_shapes(lib, T, d_out, d_in, N, M):
+    """Sizes that are not tile multiples (tiles are 128 x 256 x 128 bytes)."""
+    w = synth.trimodal_weight(d_out, d_in, seed=3, tensor_id=T)
+    x = synth.activations(T, d_in, seed=3, tensor_id=100 + T, outlier_frac=0.01)
+    dy = synth.grad_output(T, d_out, seed=3, tensor_id=200 + T)
+    _full_parity(lib, w, x, dy, N, M)
+
+
+@pytest.mark.parametrize("N,M", [(8, 8), (6, 8), (4, 8), (2, 8), (2, 4), (1, 4), (3, 4)])
+def test_mask_quant_sweep_with_ties(lib, N, M):
+    """Exact |W| ties straddling the top-N boundary keep the lower index."""
+    w = synth.trimodal_weight(384, 512, seed=4, tensor_id=N * 10 + M)
+    if N < M:
+        w = synth.with_boundary_ties(w, N, M, seed=4, frac=0.05, all_equal_groups=16)
+    from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer
+    L = SparseBitLinearLayer(_dev(w), N, M, keep_mask=True)
+    L.weight_step()
+    lib.sbl_check()
+    weff, gamma, keep = oracle.effective_weight(synth.bits(w), N, M)
+    assert np.array_equal(_unpack_mask(L.mask_bits.cpu().numpy()), keep)
+    assert L.gamma.item() == float(gamma)
+    assert np.array_equal(L.W_eff.cpu().numpy(), weff)
+
+
+def test_gamma_exact_on_extreme_magnitudes(lib):
+    """Magnitudes outside the fast window (subnormal, tiny, >= 2) and a
+    sum that naive fp32/fp64 accumulation would round differently."""
+    vals = torch.full((64, 64), 0.0)
+    vals[0, :8] = torch.tensor([1.0, 2.0 ** -53, 2.0 ** -53, 3.0e-39, 1.0e-36, 300.0, -4096.0, 2.0 ** -40])
+    vals[1:] = torch.randn(63, 64) * 0.02
+    w = vals.to(torch.bfloat16)
+    from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer
+    L = SparseBitLinearLayer(_dev(w), 6, 8)
+    L.weight_step()
+    lib.sbl_check()
+    weff, gamma, _ = oracle.effective_weight(synth.bits(w), 6, 8)
+    assert L.gamma.item() == float(gamma)
+    assert np.array_equal(L.W_eff.cpu().numpy(), weff)
+
+
+def test_dw_split_k_and_accumulate(lib):
+    """Small d_out (k/v-like) takes the split-K path with atomics; the
+    accumulate flag adds into an existing gradient."""
+    T, d_out, d_in = 1000, 128, 512
+    w = synth.normal_weight(d_out, d_in, seed=5)
+    x = synth.activations(T, d_in, seed=5)
+    dy = synth.grad_output(T, d_out, seed=5)
+    prior = torch.randn(d_out, d_in, generator=torch.Generator().manual_seed(5))
+    g = Layer(lib, w, x, dy, 6, 8, accumulate=prior)
+    ref = oracle.backward_dw(synth.bits(dy), synth.bits(x)) + prior.numpy()
+    _check_bwd(g.dW.cpu().numpy(), ref, "dW accumulate")
+
+
+def test_zero_activation_row(lib):
+    """An all-zero token quantises to zeros with amax = 1e-5 and gives y = 0."""
+    w = synth.normal_weight(64, 128, seed=6)
+    x = synth.activations(5, 128, seed=6).to(torch.float32)
+    x[2] = 0.0
+    x = x.to(torch.bfloat16)
+    dy = synth.grad_output(5, 64, seed=6)
+    g, ref = _full_parity(lib, w, x, dy, 6, 8)
+    assert (g.Xq[2] == 0).all() and g.amax[2].item() == np.float32(1e-5) and (g.Y[2] == 0).all()
+
+
+def test_argument_errors_return_status(lib):
+    import semi_structured_sparsity_step_b200._binding as B
+    ll = B.load()
+    W = torch.zeros(8, 16, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(8, 16, dtype=torch.int8, device="cuda")
+    g = torch.zeros(1, device="cuda")
+    ws = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    assert ll.sbl_mask_quant(W.data_ptr(), 8, 16, 7, 6, out.data_ptr(), None, None, g.data_ptr(), ws.data_ptr(),
+                             ws.numel(), s) == 1  # M not in {4, 8}
+    assert ll.sbl_mask_quant(W.data_ptr(), 8, 12, 6, 8, out.data_ptr(), None, None, g.data_ptr(), ws.data_ptr(),
+                             ws.numel(), s) == 2  # d_in % 16
+    assert ll.sbl_mask_quant(W.data_ptr() + 2, 8, 16, 6, 8, out.data_ptr(), None, None, g.data_ptr(),
+                             ws.data_ptr(), ws.numel(), s) == 3  # misaligned
+    assert ll.sbl_mask_quant(W.data_ptr(), 8, 16, 6, 8, out.data_ptr(), None, None, g.data_ptr(), ws.data_ptr(),
+                             16, s) == 5  # workspace too small
+    lib.sbl_check()
+
+
+# ------------------------------------------------------------------ pack / GEMV
+@pytest.mark.parametrize("N,M", [(6, 8), (2, 4), (8, 8), (4, 8), (1, 8), (3, 4)])
+def test_pack_bytes_bit_exact(lib, N, M):
+    d_out, d_in = 24, 272
+    w = synth.trimodal_weight(d_out, d_in, seed=7, tensor_id=N * 10 + M)
+    weff, _, _ = oracle.effective_weight(synth.bits(w), N, M)
+    nbytes = lib.sbl_packed_bytes(d_out, d_in, N, M)
+    assert nbytes == oracle.packed_layout(d_out, d_in, N, M)[2]
+    packed = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device="cuda")
+    lib.sbl_pack(torch.from_numpy(weff).cuda(), d_out, d_in, N, M, packed, nbytes)
+    lib.sbl_check()
+    assert np.array_equal(packed.cpu().numpy(), oracle.pack(weff, N, M))
+
+
+def test_pack_rejects_too_many_nonzeros(lib):
+    weff = torch.ones(8, 16, dtype=torch.int8, device="cuda")
+    nbytes = lib.sbl_packed_bytes(8, 16, 6, 8)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    lib.sbl_pack(weff, 8, 16, 6, 8, packed, nbytes)
+    with pytest.raises(lib.SblError) as e:
+        lib.sbl_check()
+    assert e.value.status == 8
+    lib.sbl_check()  # the latched error was cleared
+
+
+@pytest.mark.parametrize("batch", [1, 3, 8, 16])
+@pytest.mark.parametrize("N,M", [(6, 8), (2, 4), (8, 8)])
+def test_gemv_packed_parity(lib, batch, N, M):
+    d_out, d_in = 520, 2064
+    w = synth.trimodal_weight(d_out, d_in, seed=8, tensor_id=batch)
+    weff, gamma, _ = oracle.effective_weight(synth.bits(w), N, M)
+    x = synth.activations(batch, d_in, seed=8, tensor_id=100 + batch)
+    xq, amax = oracle.act_quant(synth.bits(x))
+    nbytes = lib.sbl_packed_bytes(d_out, d_in, N, M)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    lib.sbl_pack(torch.from_numpy(weff).cuda(), d_out, d_in, N, M, packed, nbytes)
+    Y = torch.empty(batch, d_out, dtype=torch.float32, device="cuda")
+    g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+    lib.sbl_gemv_packed(torch.from_numpy(xq).cuda(), torch.from_numpy(amax).cuda(), batch, packed, g, d_in, d_out,
+                        N, M, Y)
+    lib.sbl_check()
+    ref = oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax)
+    assert np.array_equal(Y.cpu().numpy(), ref)

@@ -1,0 +1,78 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every entry point
+that include/sbl.h declares, and rejects bad arguments on the host before
+touching CUDA (no GPU is needed for any of this)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sbl.h")
+
+
+@pytest.fixture(scope="module")
+def cl():
+    from semi_structured_sparsity_step_b200 import build
+    build.build()
+    from semi_structured_sparsity_step_b200 import _binding
+    return _binding.load()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sbl_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_north_star_calls():
+    names = _declared()
+    for n in ["sbl_mask_quant", "sbl_act_quant", "sbl_forward", "sbl_backward", "sbl_pack", "sbl_gemv_packed",
+              "sbl_check", "sbl_status_string", "sbl_packed_bytes"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(cl):
+    from semi_structured_sparsity_step_b200._binding import SIGNATURES
+    for n in _declared():
+        assert hasattr(cl, n), n
+        assert n in SIGNATURES, n
+
+
+def test_status_strings(cl):
+    from semi_structured_sparsity_step_b200 import _binding as B
+    for code, name in B.STATUS.items():
+        assert B.sbl_status_string(code) == name
+    assert B.sbl_status_string(99) == "SBL_ERR_UNKNOWN"
+
+
+def test_host_validation_without_gpu(cl):
+    al = 1 << 12  # fake, 16-byte aligned addresses: never dereferenced on these paths
+    # bad N:M
+    assert cl.sbl_mask_quant(al, 8, 16, 0, 8, al, None, None, al, al * 4, 1 << 20, None) == 1
+    assert cl.sbl_mask_quant(al, 8, 16, 5, 6, al, None, None, al, al * 4, 1 << 20, None) == 1
+    assert cl.sbl_mask_quant(al, 8, 16, 9, 8, al, None, None, al, al * 4, 1 << 20, None) == 1
+    # shapes
+    assert cl.sbl_mask_quant(al, 8, 24, 6, 8, al, None, None, al, al * 4, 1 << 20, None) == 2
+    assert cl.sbl_mask_quant(al, 12, 16, 6, 8, al, None, None, al, al * 4, 1 << 20, None) == 2
+    assert cl.sbl_act_quant(al, -1, 16, al, al, None) == 2
+    assert cl.sbl_forward(al, al, al, al, 4, 20, 8, al, None, None) == 2
+    assert cl.sbl_gemv_packed(al, al, 17, al, al, 16, 8, 6, 8, al, None) == 2
+    # null and misaligned pointers
+    assert cl.sbl_mask_quant(None, 8, 16, 6, 8, al, None, None, al, al * 4, 1 << 20, None) == 1
+    assert cl.sbl_act_quant(al + 8, 4, 16, al, al, None) == 3
+    assert cl.sbl_forward(al, al, al + 4, al, 4, 16, 8, al, None, None) == 3
+    assert cl.sbl_mask_quant(al, 8, 16, 6, 8, al, None, None, al, al + 16, 1 << 20, None) == 3
+    # workspace and packed buffer too small
+    assert cl.sbl_mask_quant(al, 8, 16, 6, 8, al, None, None, al, al * 4, 8, None) == 5
+    assert cl.sbl_pack(al, 8, 16, 6, 8, al, 4, None) == 5
+    # empty work is a no-op that needs no device
+    assert cl.sbl_act_quant(al, 0, 16, al, al, None) == 0
+    assert cl.sbl_forward(al, al, al, al, 0, 16, 8, al, None, None) == 0
+
+
+def test_packed_bytes_matches_format(cl):
+    import oracle
+    for (d_out, d_in, N, M) in [(8, 16, 6, 8), (24, 272, 2, 4), (2048, 11008, 6, 8), (16, 64, 8, 8)]:
+        assert cl.sbl_packed_bytes(d_out, d_in, N, M) == oracle.packed_layout(d_out, d_in, N, M)[2]
+    assert cl.sbl_packed_bytes(8, 24, 6, 8) == 0  # invalid shape
