@@ -147,7 +147,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except (OSError, ValueError):
@@ -187,7 +187,7 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- CPU oracle timing
-def oracle_sample(ls, T_full, tokens=16, seed=0):
+def oracle_sample(ls, T_full, tokens=128, seed=0):
     """Time the oracle as it stands on a bounded sample of the workload and
     extrapolate to one full step: the weight side of the q projection scaled
     by parameter count, the token side of all projections on `tokens` tokens
@@ -255,7 +255,7 @@ def traffic_for(kernel_key):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sbl", "reference"], default="sbl")
     ap.add_argument("--e2e-steps", type=int, default=2)
