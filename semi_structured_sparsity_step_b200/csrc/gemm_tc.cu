@@ -61,105 +61,118 @@ struct Cfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  static constexpr uint32_t TMEM_COLS = BN;
+  static constexpr int EPI_WARP_FLOATS = 32 * 33;  // 32 x 32 fp32 transpose tile, padded rows
+  static constexpr int EPI_BYTES = 4 * EPI_WARP_FLOATS * 4;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulator buffers
   static constexpr uint32_t IDESC = instr_desc(kI8, BM, BN, kAMN, kBMN);
 };
 
+// Work item -> (m block, n block, k split).  n varies fastest, so the CTAs
+// that run at the same time share the weight-side (B) tiles and each A row
+// block is fetched from HBM once.
+struct Sched {
+  int Mt, Nt, splits, total;
+  __device__ __forceinline__ void item(int w, int& mb, int& nb, int& sp) const {
+    const int per = Mt * Nt;
+    sp = w / per;
+    const int r = w - sp * per;
+    mb = r / Nt;
+    nb = r - mb * Nt;
+  }
+};
+
+// Epilogue of one 32 x 32 chunk held one row per lane (r[j] = column j).
+// Phase 1 applies the scale in that layout and writes the chunk into a padded
+// shared tile; phase 2 reads it back four rows per instruction, so every
+// global access of the warp covers four whole 128-byte row segments.
 template <int EPI>
-__device__ __forceinline__ void store_chunk(const GemmArgs& a, int row, int col0, const uint32_t (&r)[32],
-                                            float scale) {
-  float* orow = a.out + static_cast<long long>(row) * a.ldo;
-  float v[32];
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, float* tile, int row0, int col0, int lane,
+                                               const uint32_t (&r)[32], float scale) {
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
+    float v;
     if constexpr (EPI == kEpiFwd) {
-      v[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scale);
+      v = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scale);
     } else if constexpr (EPI == kEpiDx) {
-      v[j] = __fmul_rn(scale, __uint_as_float(r[j]));
+      v = __fmul_rn(scale, __uint_as_float(r[j]));
     } else {
-      v[j] = __uint_as_float(r[j]);
+      v = __uint_as_float(r[j]);
     }
-  }
-  const bool full = col0 + 32 <= a.N;
-  if constexpr (EPI == kEpiDw) {
-    if (a.atomic_out) {
-      if (full) {
-#pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          atomicAdd(reinterpret_cast<float4*>(orow + col0 + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
-      } else {
-        for (int j = 0; j < 32 && col0 + j < a.N; ++j) atomicAdd(orow + col0 + j, v[j]);
-      }
-      return;
-    }
-    if (a.accumulate) {
-      if (full) {
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          float4 o = *reinterpret_cast<const float4*>(orow + col0 + j);
-          o.x = __fadd_rn(o.x, v[j]);
-          o.y = __fadd_rn(o.y, v[j + 1]);
-          o.z = __fadd_rn(o.z, v[j + 2]);
-          o.w = __fadd_rn(o.w, v[j + 3]);
-          *reinterpret_cast<float4*>(orow + col0 + j) = o;
-        }
-      } else {
-        for (int j = 0; j < 32 && col0 + j < a.N; ++j) orow[col0 + j] = __fadd_rn(orow[col0 + j], v[j]);
-      }
-      return;
-    }
-  }
-  if (full) {
-#pragma unroll
-    for (int j = 0; j < 32; j += 4)
-      *reinterpret_cast<float4*>(orow + col0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-  } else {
-    for (int j = 0; j < 32 && col0 + j < a.N; ++j) orow[col0 + j] = v[j];
+    tile[lane * 33 + j] = v;
   }
   if constexpr (EPI == kEpiFwd) {
-    if (a.acc_out != nullptr) {
-      int32_t* arow = a.acc_out + static_cast<long long>(row) * a.ldo;
-      if (full) {
+    if (a.acc_out != nullptr && row0 + lane < a.M) {
+      int32_t* arow = a.acc_out + static_cast<long long>(row0 + lane) * a.ldo + col0;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<int4*>(arow + col0 + j) = make_int4(static_cast<int>(r[j]), static_cast<int>(r[j + 1]),
-                                                                static_cast<int>(r[j + 2]), static_cast<int>(r[j + 3]));
-      } else {
-        for (int j = 0; j < 32 && col0 + j < a.N; ++j) arow[col0 + j] = static_cast<int>(r[j]);
-      }
+      for (int j = 0; j < 32; j += 4)
+        if (col0 + j < a.N)
+          *reinterpret_cast<int4*>(arow + j) = make_int4(static_cast<int>(r[j]), static_cast<int>(r[j + 1]),
+                                                         static_cast<int>(r[j + 2]), static_cast<int>(r[j + 3]));
     }
   }
+  __syncwarp();
+  const int cq = (lane & 7) * 4;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int rr = it * 4 + (lane >> 3);
+    const int grow = row0 + rr;
+    const int gcol = col0 + cq;
+    if (grow < a.M && gcol < a.N) {  // N % 8 == 0: a float4 is either all in or all out
+      const float* t = tile + rr * 33 + cq;
+      float4 v = make_float4(t[0], t[1], t[2], t[3]);
+      float* dst = a.out + static_cast<long long>(grow) * a.ldo + gcol;
+      if constexpr (EPI == kEpiDw) {
+        if (a.atomic_out) {
+          atomicAdd(reinterpret_cast<float4*>(dst), v);
+          continue;
+        }
+        if (a.accumulate) {
+          const float4 o = *reinterpret_cast<const float4*>(dst);
+          v.x = __fadd_rn(o.x, v.x);
+          v.y = __fadd_rn(o.y, v.y);
+          v.z = __fadd_rn(o.z, v.z);
+          v.w = __fadd_rn(o.w, v.w);
+        }
+      }
+      *reinterpret_cast<float4*>(dst) = v;
+    }
+  }
+  __syncwarp();
 }
 
+// Persistent kernel: one CTA per SM walks the work items blockIdx.x,
+// blockIdx.x + gridDim.x, ...  The shared-memory ring and its phases run on
+// across items; the accumulator alternates between two TMEM buffers so the
+// epilogue of one item overlaps the tensor-core work of the next.
 template <bool kI8, bool kAMN, bool kBMN, int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs args) {
+                   const GemmArgs args, const Sched sched) {
   using C = Cfg<kI8, kAMN, kBMN, BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  float* epi_tiles = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* accum = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  uint64_t* tfull = empty + STAGES;  // [2] accumulator buffer ready for the epilogue
+  uint64_t* tempty = tfull + 2;      // [2] accumulator buffer drained by the epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM;
-  const int n0 = blockIdx.x * BN;
   const int KB = (args.K + C::BK - 1) / C::BK;
-  const int kb0 = blockIdx.z * args.kb_per_split;
-  const int kb1 = min(KB, kb0 + args.kb_per_split);
-  const int nk = kb1 - kb0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -176,77 +189,115 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % STAGES;
-        const uint32_t round = static_cast<uint32_t>(i / STAGES);
-        if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, args.err)) break;
-        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-        uint8_t* sa = smem + s * C::STAGE_BYTES;
-        uint8_t* sb = sa + C::A_BYTES;
-        const int kc = (kb0 + i) * C::BK;
-        if constexpr (!kAMN) {
-          tma_load_2d(sa, &tmA, &full[s], kc, m0);
-        } else {
+      int it = 0;  // k-blocks issued by this CTA so far (position in the stage ring)
+      bool ok = true;
+      for (int w = blockIdx.x; w < sched.total && ok; w += gridDim.x) {
+        int mb, nb, sp;
+        sched.item(w, mb, nb, sp);
+        const int kb0 = sp * args.kb_per_split;
+        const int kb1 = min(KB, kb0 + args.kb_per_split);
+        const int m0 = mb * BM, n0 = nb * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t round = static_cast<uint32_t>(it / STAGES);
+          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+          uint8_t* sa = smem + s * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          const int kc = kb * C::BK;
+          if constexpr (!kAMN) {
+            tma_load_2d(sa, &tmA, &full[s], kc, m0);
+          } else {
 #pragma unroll
-          for (int c = 0; c < BM / 64; ++c) tma_load_2d(sa + c * C::BK * 128, &tmA, &full[s], m0 + 64 * c, kc);
-        }
-        if constexpr (!kBMN) {
-          tma_load_2d(sb, &tmB, &full[s], kc, n0);
-        } else {
+            for (int c = 0; c < BM / 64; ++c) tma_load_2d(sa + c * C::BK * 128, &tmA, &full[s], m0 + 64 * c, kc);
+          }
+          if constexpr (!kBMN) {
+            tma_load_2d(sb, &tmB, &full[s], kc, n0);
+          } else {
 #pragma unroll
-          for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * C::BK * 128, &tmB, &full[s], n0 + 64 * c, kc);
+            for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * C::BK * 128, &tmB, &full[s], n0 + 64 * c, kc);
+          }
+          ++it;
         }
-        issued = i + 1;
       }
-      if (*abort_flag) {
+      if (!ok) {
         // Let the copies already in flight land before the block exits.
-        for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+        for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i)
           mbar_wait(&full[i % STAGES], static_cast<uint32_t>(i / STAGES) & 1u, nullptr, args.err);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % STAGES;
-        const uint32_t round = static_cast<uint32_t>(i / STAGES);
-        if (!mbar_wait(&full[s], round & 1u, abort_flag, args.err)) break;
+      int it = 0, t = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < sched.total && ok; w += gridDim.x, ++t) {
+        int mb, nb, sp;
+        sched.item(w, mb, nb, sp);
+        const int kb0 = sp * args.kb_per_split;
+        const int kb1 = min(KB, kb0 + args.kb_per_split);
+        const int b = t & 1;
+        if (!mbar_wait(&tempty[b], (static_cast<uint32_t>(t >> 1) & 1u) ^ 1u, abort_flag, args.err)) break;
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
-        const uint32_t sb = sa + C::A_BYTES;
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t round = static_cast<uint32_t>(it / STAGES);
+          if (!mbar_wait(&full[s], round & 1u, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < C::BK / C::UK; ++kk) {
-          const uint64_t adesc = kAMN ? smem_desc_sw128(sa + kk * C::UK * 128, C::BK * 128, 1024)
-                                      : smem_desc_sw128(sa + kk * 32, 16, 1024);
-          const uint64_t bdesc = kBMN ? smem_desc_sw128(sb + kk * C::UK * 128, C::BK * 128, 1024)
-                                      : smem_desc_sw128(sb + kk * 32, 16, 1024);
-          umma<kI8>(tmem_base, adesc, bdesc, C::IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < C::BK / C::UK; ++kk) {
+            const uint64_t adesc = kAMN ? smem_desc_sw128(sa + kk * C::UK * 128, C::BK * 128, 1024)
+                                        : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bdesc = kBMN ? smem_desc_sw128(sb + kk * C::UK * 128, C::BK * 128, 1024)
+                                        : smem_desc_sw128(sb + kk * 32, 16, 1024);
+            umma<kI8>(d_tmem, adesc, bdesc, C::IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          ++it;
         }
-        umma_commit(&empty[s]);
+        umma_commit(&tfull[b]);  // fires when this item's MMAs are done (also on abort)
       }
-      umma_commit(accum);
     }
   } else {
-    const bool ok = mbar_wait(accum, 0u, abort_flag, args.err);
-    tc_fence_after();
-    if (ok && !*abort_flag) {
-      const int q = warp & 3;
-      const int row = m0 + 32 * q + lane;
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    float* tile = epi_tiles + q * C::EPI_WARP_FLOATS;
+    int t = 0;
+    for (int w = blockIdx.x; w < sched.total; w += gridDim.x, ++t) {
+      int mb, nb, sp;
+      sched.item(w, mb, nb, sp);
+      const int b = t & 1;
+      if (!mbar_wait(&tfull[b], static_cast<uint32_t>(t >> 1) & 1u, abort_flag, args.err)) break;
+      tc_fence_after();
+      if (*abort_flag) break;
+      const int row0 = mb * BM + 32 * q;
+      const int row = row0 + lane;
       float scale = 0.0f;
       if constexpr (EPI == kEpiFwd) {
         if (row < args.M) scale = __fmul_rn(*args.gamma, __fdiv_rn(args.amax[row], 127.0f));
       } else if constexpr (EPI == kEpiDx) {
         scale = *args.gamma;
       }
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b * BN);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
-        const int col0 = n0 + 32 * c;
+        const int col0 = nb * BN + 32 * c;
         if (col0 >= args.N) break;  // warp-uniform
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(32 * c), r);
+        tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(32 * c), r);
         tmem_ld_wait();
-        if (row < args.M) store_chunk<EPI>(args, row, col0, r, scale);
+        epilogue_chunk<EPI>(args, tile, row0, col0, lane, r, scale);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[b]);
     }
   }
   tc_fence_before();
@@ -293,14 +344,19 @@ bool make_tmap(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint
 }
 
 template <bool kI8, bool kAMN, bool kBMN, int BN, int STAGES, int EPI>
-cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int splits,
+cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int splits, int num_sms,
                 cudaStream_t stream) {
   using C = Cfg<kI8, kAMN, kBMN, BN, STAGES>;
   auto kern = tc_gemm_kernel<kI8, kAMN, kBMN, BN, STAGES, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM, splits);
-  kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(ta, tb, a);
+  Sched sc;
+  sc.Mt = (a.M + BM - 1) / BM;
+  sc.Nt = (a.N + BN - 1) / BN;
+  sc.splits = splits;
+  sc.total = sc.Mt * sc.Nt * splits;
+  const int grid = sc.total < num_sms ? sc.total : num_sms;
+  kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(ta, tb, a, sc);
   return cudaGetLastError();
 }
 
@@ -312,7 +368,6 @@ constexpr int kStages = 4;
 cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
                            int d_in, int d_out, float* Y, int32_t* acc, cudaStream_t stream, int num_sms,
                            uint32_t* err) {
-  (void)num_sms;
   if (T == 0 || d_out == 0) return cudaSuccess;
   if (d_in == 0) {
     cudaError_t e = cudaMemsetAsync(Y, 0, sizeof(float) * static_cast<size_t>(T) * d_out, stream);
@@ -334,7 +389,7 @@ cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_
   a.amax = amax;
   a.gamma = gamma;
   a.err = err;
-  return run<true, false, false, kBN, kStages, kEpiFwd>(ta, tb, a, 1, stream);
+  return run<true, false, false, kBN, kStages, kEpiFwd>(ta, tb, a, 1, num_sms, stream);
 }
 
 cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf16, const float* gamma, int T,
@@ -358,7 +413,7 @@ cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf1
       a.ldo = d_in;
       a.gamma = gamma;
       a.err = err;
-      e = run<false, false, true, kBN, kStages, kEpiDx>(ta, tb, a, 1, stream);
+      e = run<false, false, true, kBN, kStages, kEpiDx>(ta, tb, a, 1, num_sms, stream);
     }
     if (e != cudaSuccess) return e;
   }
@@ -392,7 +447,7 @@ cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf1
       e = cudaMemsetAsync(dW, 0, sizeof(float) * static_cast<size_t>(d_out) * d_in, stream);
       if (e != cudaSuccess) return e;
     }
-    e = run<false, true, true, kBN, kStages, kEpiDw>(ta, tb, a, splits, stream);
+    e = run<false, true, true, kBN, kStages, kEpiDw>(ta, tb, a, splits, num_sms, stream);
   }
   return e;
 }

@@ -19,14 +19,15 @@
 //      the per-block window sums in 128 bits, folds everything into one
 //      320-bit integer (unit 2^-133), rounds it once to fp64 (nearest-even),
 //      divides by n in fp64 and rounds to fp32.  The result does not depend
-//      on the order of the additions.
-//   2. ternary_mask_kernel: one thread per 8 weights (one uint4).  The
-//      ternary code only depends on whether fp32(|w| / den) > 0.5, which is
-//      monotone in |w|, so each block first finds (binary search with the
-//      IEEE divide) the largest bf16 magnitude that still maps to 0, then
-//      every weight is one integer compare.  The mask ranks the 15-bit
-//      magnitudes with the position as tie-break (lower index wins), using
-//      pairwise compares in registers.
+//      on the order of the additions.  The ternary code only depends on
+//      whether fp32(|w| / den) > 0.5 (den = fp32(gamma + 1e-5)), which is
+//      monotone in |w|, so the same block also finds, by binary search with
+//      the IEEE divide, the largest bf16 magnitude that still maps to 0 and
+//      leaves it in the workspace.
+//   2. ternary_mask_kernel: one thread per 8 weights (one uint4); each
+//      ternary code is one integer compare against that threshold.  The
+//      mask ranks the 15-bit magnitudes with the position as tie-break
+//      (lower index wins), using pairwise compares in registers.
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -67,30 +68,27 @@ __device__ void bigint_add_shifted(uint32_t* limbs, uint64_t v, int shift) {
   }
 }
 
-// Bit `pos` of the 320-bit integer (0 for pos < 0).
-__device__ __forceinline__ uint32_t bigint_bit(const uint32_t* limbs, int pos) {
-  if (pos < 0) return 0u;
-  return (limbs[pos >> 5] >> (pos & 31)) & 1u;
-}
-
 // Correctly rounded (nearest-even) fp64 value of limbs * 2^-133.
 __device__ double bigint_to_double(const uint32_t* limbs) {
-  int top = -1;
-  for (int i = kGammaLimbs - 1; i >= 0; --i) {
-    if (limbs[i] != 0u) {
-      top = 32 * i + (31 - __clz(limbs[i]));
-      break;
-    }
-  }
-  if (top < 0) return 0.0;
-  // 53 significant bits [top-52, top], then the rounding bit and the sticky bits.
-  uint64_t mant = 0;
-  for (int b = top; b >= top - 52; --b) mant = (mant << 1) | bigint_bit(limbs, b);
-  const uint32_t round_bit = bigint_bit(limbs, top - 53);
-  uint32_t sticky = 0;
-  for (int b = top - 54; b >= 0 && !sticky; --b) sticky |= bigint_bit(limbs, b);
+  int L = kGammaLimbs - 1;
+  while (L >= 0 && limbs[L] == 0u) --L;
+  if (L < 0) return 0.0;
+  const int top = 32 * L + (31 - __clz(limbs[L]));  // index of the leading one
+  // 96-bit window of limbs L, L-1, L-2 (missing limbs read as 0).
+  const uint32_t l1 = L >= 1 ? limbs[L - 1] : 0u;
+  const uint32_t l2 = L >= 2 ? limbs[L - 2] : 0u;
+  const unsigned __int128 v = (static_cast<unsigned __int128>(limbs[L]) << 64) |
+                              (static_cast<unsigned __int128>(l1) << 32) | l2;
+  const int p = 64 + (31 - __clz(limbs[L]));        // leading one inside the window
+  const int sh = p - 63;                             // 1..32
+  const uint64_t mant64 = static_cast<uint64_t>(v >> sh);  // bits [top-63, top]
+  bool sticky = (v & ((static_cast<unsigned __int128>(1) << sh) - 1)) != 0;
+  for (int i = 0; i < L - 2; ++i) sticky |= limbs[i] != 0u;
+  uint64_t mant = mant64 >> 11;                      // 53 bits
+  const uint32_t rest = static_cast<uint32_t>(mant64 & 0x7FFu);
+  sticky |= (rest & 0x3FFu) != 0u;
   int exp2 = top - 52;
-  if (round_bit && (sticky || (mant & 1ull))) {
+  if ((rest & 0x400u) && (sticky || (mant & 1ull))) {
     mant += 1;
     if (mant == (1ull << 53)) {
       mant >>= 1;
@@ -98,6 +96,18 @@ __device__ double bigint_to_double(const uint32_t* limbs) {
     }
   }
   return scalbn(static_cast<double>(mant), exp2 - 133);
+}
+
+// Largest bf16 magnitude pattern b (0 <= b < 0x7F80) with fp32(bf16(b) / den) <= 0.5.
+// fp32(|w| / den) is monotone in |w|, so W_q = 0 exactly when |w|'s pattern <= b.
+__device__ uint32_t zero_threshold_bits(float den) {
+  uint32_t lo = 0u, hi = 0x7F80u;  // cond(lo) holds; cond(hi) fails (inf)
+  while (hi - lo > 1u) {
+    const uint32_t mid = (lo + hi) >> 1;
+    const float v = __uint_as_float(mid << 16);
+    if (__fdiv_rn(v, den) <= 0.5f) lo = mid; else hi = mid;
+  }
+  return lo;
 }
 
 __global__ void __launch_bounds__(kGammaThreads) gamma_reduce_kernel(const uint4* __restrict__ W, size_t n_vec,
@@ -147,6 +157,7 @@ __global__ void __launch_bounds__(kGammaThreads) gamma_reduce_kernel(const uint4
   }
   s_lo[threadIdx.x] = lo;
   s_hi[threadIdx.x] = hi;
+  sbucket[threadIdx.x] = __ldcg(&ws->bucket[threadIdx.x]);
   __syncthreads();
   if (threadIdx.x != 0) return;
   lo = 0;
@@ -161,25 +172,14 @@ __global__ void __launch_bounds__(kGammaThreads) gamma_reduce_kernel(const uint4
   // value = m * 2^(ee-134) = m * 2^(ee-1) units of 2^-133; window sums carry 2^(96-1).
   bigint_add_shifted(limbs, lo, kWinLo - 1);
   bigint_add_shifted(limbs, hi, kWinLo - 1 + 64);
-  for (int ee = 1; ee < 256; ++ee) {
-    const uint64_t b = __ldcg(reinterpret_cast<const unsigned long long*>(&ws->bucket[ee]));
-    bigint_add_shifted(limbs, b, ee - 1);
-  }
+  for (int ee = 1; ee < 256; ++ee) bigint_add_shifted(limbs, sbucket[ee], ee - 1);
   const double total = bigint_to_double(limbs);
   const double mean = __ddiv_rn(total, static_cast<double>(n_elems));
-  *gamma_out = __double2float_rn(mean);
+  const float gamma = __double2float_rn(mean);
+  *gamma_out = gamma;
+  ws->zero_threshold = zero_threshold_bits(__fadd_rn(gamma, 1e-5f));
 }
 
-// Largest bf16 magnitude pattern b (0 <= b < 0x7F80) with fp32(bf16(b) / den) <= 0.5.
-__device__ uint32_t zero_threshold_bits(float den) {
-  uint32_t lo = 0u, hi = 0x7F80u;  // cond(lo) true; cond(hi) false (inf)
-  while (hi - lo > 1u) {
-    const uint32_t mid = (lo + hi) >> 1;
-    const float v = __uint_as_float(mid << 16);
-    if (__fdiv_rn(v, den) <= 0.5f) lo = mid; else hi = mid;
-  }
-  return lo;
-}
 
 template <int M>
 __device__ __forceinline__ void rank_keep(const uint32_t (&mag)[8], int N, uint32_t& keep_bits) {
@@ -210,14 +210,11 @@ __device__ __forceinline__ void rank_keep(const uint32_t (&mag)[8], int N, uint3
 
 template <int M>
 __global__ void __launch_bounds__(256) ternary_mask_kernel(const uint4* __restrict__ W, size_t n_vec, int N,
-                                                           const float* __restrict__ gamma,
+                                                           const GammaWorkspace* __restrict__ ws,
                                                            uint2* __restrict__ w_eff,
                                                            uint4* __restrict__ w_eff_bf16,
                                                            uint8_t* __restrict__ mask_bits) {
-  __shared__ uint32_t s_thr;
-  if (threadIdx.x == 0) s_thr = zero_threshold_bits(__fadd_rn(*gamma, 1e-5f));
-  __syncthreads();
-  const uint32_t thr = s_thr;
+  const uint32_t thr = ws->zero_threshold;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_vec;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const uint4 v = __ldg(W + i);
@@ -274,11 +271,11 @@ cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, 
   if (qblocks < 1) qblocks = 1;
   if (M == 8) {
     ternary_mask_kernel<8><<<static_cast<unsigned>(qblocks), 256, 0, stream>>>(
-        static_cast<const uint4*>(W), n_vec, N, gamma, reinterpret_cast<uint2*>(W_eff),
+        static_cast<const uint4*>(W), n_vec, N, ws, reinterpret_cast<uint2*>(W_eff),
         static_cast<uint4*>(W_eff_bf16), mask_bits);
   } else {
     ternary_mask_kernel<4><<<static_cast<unsigned>(qblocks), 256, 0, stream>>>(
-        static_cast<const uint4*>(W), n_vec, N, gamma, reinterpret_cast<uint2*>(W_eff),
+        static_cast<const uint4*>(W), n_vec, N, ws, reinterpret_cast<uint2*>(W_eff),
         static_cast<uint4*>(W_eff_bf16), mask_bits);
   }
   return cudaGetLastError();

@@ -15,7 +15,8 @@ constexpr int kGammaLimbs = 10;       // 320-bit exact sum of |W| in units of 2^
 struct GammaWorkspace {
   unsigned long long bucket[256];  // sum of 8-bit significands per biased exponent
   unsigned int ticket;             // blocks finished
-  unsigned int pad[63];
+  unsigned int zero_threshold;     // largest bf16 magnitude pattern with W_q = 0
+  unsigned int pad[62];
   unsigned long long block_window[kGammaMaxBlocks];  // per-block window sums
 };
 

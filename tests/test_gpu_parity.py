@@ -224,3 +224,20 @@ def test_gemv_packed_parity(lib, batch, N, M):
     lib.sbl_check()
     ref = oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax)
     assert np.array_equal(Y.cpu().numpy(), ref)
+
+
+def test_gamma_exact_on_log_uniform_magnitudes(lib):
+    """Magnitudes spread log-uniformly over 2^-133 .. 2^12 fill many exponent
+    buckets as well as the register window; gamma and the codes stay exact."""
+    g = torch.Generator().manual_seed(11)
+    e = torch.rand(512, 1024, generator=g) * 145.0 - 133.0
+    sign = torch.where(torch.rand(512, 1024, generator=g) < 0.5, -1.0, 1.0)
+    w = (sign * torch.exp2(e)).to(torch.bfloat16)
+    from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer
+    for N, M in [(6, 8), (2, 4)]:
+        L = SparseBitLinearLayer(_dev(w), N, M)
+        L.weight_step()
+        lib.sbl_check()
+        weff, gamma, _ = oracle.effective_weight(synth.bits(w), N, M)
+        assert L.gamma.item() == float(gamma)
+        assert np.array_equal(L.W_eff.cpu().numpy(), weff)
