@@ -40,8 +40,12 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-WORKLOAD = "qwen2.5-3b"
-T_TOKENS = 32768
+WORKLOADS = {
+    # name: (default tokens, weight distribution, outlier fraction of X channels, boundary-tie groups)
+    "qwen2.5-3b": (32768, "trimodal", 0.001, 0.0),
+    "qwen2.5-0.5b": (4096, "normal", 0.0, 0.0),
+    "qwen2.5-3b-up": (8192, "trimodal", 0.001, 0.01),
+}
 N_KEEP, M_GROUP = 6, 8
 METRIC = "Sparse-BitLinear fwd+bwd tokens/s (3B-shape, 6:8)"
 
@@ -58,13 +62,25 @@ def peaks():
 
 
 # ----------------------------------------------------------------- inputs
+def make_weight(ls, i, p):
+    _, dist, _, ties = WORKLOADS[ls.name]
+    if dist == "trimodal":
+        w = synth.trimodal_weight(p.d_out, p.d_in, seed=0, tensor_id=i)
+    else:
+        w = synth.normal_weight(p.d_out, p.d_in, seed=0, tensor_id=i)
+    if ties > 0 and N_KEEP < M_GROUP:
+        w = synth.with_boundary_ties(w, N_KEEP, M_GROUP, seed=0, tensor_id=300 + i, frac=ties)
+    return w
+
+
 def make_inputs(ls, T, seed, device):
     """Seeded synthetic tensors for one step, on `device` (CPU pinned or cuda)."""
     W, X, dY = {}, {}, {}
+    outl = WORKLOADS[ls.name][2]
     for i, p in enumerate(ls.projections):
-        W[p.name] = synth.trimodal_weight(p.d_out, p.d_in, seed=0, tensor_id=i)  # replicated weights
+        W[p.name] = make_weight(ls, i, p)  # replicated across ranks
     for j, (name, d_in) in enumerate(ls.inputs.items()):
-        X[name] = synth.activations(T, d_in, seed=seed, tensor_id=100 + j, outlier_frac=0.001)
+        X[name] = synth.activations(T, d_in, seed=seed, tensor_id=100 + j, outlier_frac=outl)
     for i, p in enumerate(ls.projections):
         dY[p.name] = synth.grad_output(T, p.d_out, seed=seed, tensor_id=200 + i)
     if device == "pinned":
@@ -90,7 +106,8 @@ class Step:
         self.Y = {p.name: torch.empty(T, p.d_out, dtype=torch.float32, device=dev) for p in ls.projections}
         self.dX = {p.name: torch.empty(T, p.d_in, dtype=torch.float32, device=dev) for p in ls.projections}
         self.dW = {p.name: torch.empty(p.d_out, p.d_in, dtype=torch.float32, device=dev) for p in ls.projections}
-        self.kernels_per_step = 2 * 7 + 4 + 7 + 7 + 7
+        n_p, n_x = len(ls.projections), len(ls.inputs)
+        self.kernels_per_step = 2 * n_p + n_x + 3 * n_p
 
     def run(self, stream, ev=None):
         """Enqueue one step.  With `ev` (dict name -> list), record event pairs per call."""
@@ -194,18 +211,18 @@ def oracle_sample(ls, T_full, tokens=128, seed=0):
     scaled to T_full tokens."""
     import oracle
     q = ls.projections[0]
-    wq = synth.bits(synth.trimodal_weight(q.d_out, q.d_in, seed=0, tensor_id=0))
+    wq = synth.bits(make_weight(ls, 0, q))
     t0 = time.perf_counter()
     oracle.effective_weight(wq, N_KEEP, M_GROUP)
     t_w = time.perf_counter() - t0
     weight_side = t_w * ls.params / (q.d_out * q.d_in)
-    xs = {n: synth.bits(synth.activations(tokens, d, seed=seed, tensor_id=100 + j, outlier_frac=0.001))
+    outl = WORKLOADS[ls.name][2]
+    xs = {n: synth.bits(synth.activations(tokens, d, seed=seed, tensor_id=100 + j, outlier_frac=outl))
           for j, (n, d) in enumerate(ls.inputs.items())}
     t_tok = 0.0
     weffs = {}
     for i, p in enumerate(ls.projections):
-        w = synth.bits(synth.trimodal_weight(p.d_out, p.d_in, seed=0, tensor_id=i))
-        weffs[p.name] = oracle.effective_weight(w, N_KEEP, M_GROUP)
+        weffs[p.name] = oracle.effective_weight(synth.bits(make_weight(ls, i, p)), N_KEEP, M_GROUP)
     for n in ls.inputs:
         t0 = time.perf_counter()
         oracle.act_quant(xs[n])
@@ -226,9 +243,9 @@ def oracle_sample(ls, T_full, tokens=128, seed=0):
         cores = max([1] + [d.get("num_threads", 1) for d in threadpool_info()])
     except Exception:  # pragma: no cover
         cores = 1
-    sample = (f"oracle weight side on q ({q.d_out}x{q.d_in}) scaled x{ls.params / (q.d_out * q.d_in):.2f} by "
-              f"parameter count + token side of all 7 projections on {tokens} tokens scaled x{T_full // tokens}; "
-              f"extrapolated")
+    sample = (f"oracle weight side on {q.name} ({q.d_out}x{q.d_in}) scaled x{ls.params / (q.d_out * q.d_in):.2f} "
+              f"by parameter count + token side of all {len(ls.projections)} projections on {tokens} tokens "
+              f"scaled x{T_full // tokens}; extrapolated")
     return step_s, cores, sample, t_w + t_tok
 
 
@@ -260,18 +277,23 @@ def main():
     ap.add_argument("--impl", choices=["sbl", "reference"], default="sbl")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen2.5-3b")
+    ap.add_argument("--tokens", type=int, default=0, help="tokens per step (0: the workload's default)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    ls = synth.layer_set(WORKLOAD)
-    T = T_TOKENS
-    config = {"workload": f"{WORKLOAD} layer set (q/o 2048x2048, k/v 256x2048, gate/up 11008x2048, "
-                          f"down 2048x11008), {T} tokens (16 x 2048), N:M {N_KEEP}:{M_GROUP}, trimodal bf16 "
-                          f"master W, X ~ N(0,1) with 0.1% outlier channels x10, dY ~ N(0,1)",
+    ls = synth.layer_set(args.workload)
+    T = args.tokens or WORKLOADS[args.workload][0]
+    dist_name, outl, ties = WORKLOADS[args.workload][1:]
+    shapes = ", ".join(f"{p.name} {p.d_out}x{p.d_in}" for p in ls.projections)
+    config = {"workload": f"{args.workload} ({shapes}), {T} tokens, N:M {N_KEEP}:{M_GROUP}, {dist_name} bf16 "
+                          f"master W" + (f" with {ties:.0%} boundary-tie groups" if ties else "") +
+                          f", X ~ N(0,1)" + (f" with {outl:.1%} outlier channels x10" if outl else "") +
+                          ", dY ~ N(0,1)",
               "tokens_per_step": T, "params": ls.params, "nm": f"{N_KEEP}:{M_GROUP}",
-              "l2": "inputs larger than L2 (~11 GB per step), no flush", "parallelism": f"dp{args.gpus} replicas"}
+              "l2": "per-step working set larger than L2, no flush", "parallelism": f"dp{args.gpus} replicas"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -359,7 +381,7 @@ def main():
                 h.copy_(d, non_blocking=True)
     e1.record(stream)
     stream.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    e2e_ms = e0.elapsed_time(e1) / max(1, args.e2e_steps)
     if dist is not None:
         t = torch.tensor([e2e_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

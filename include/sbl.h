@@ -66,6 +66,14 @@ const char* sbl_status_string(int status);
 /* Library ABI version (major * 100 + minor). */
 int sbl_version(void);
 
+/* Select the tensor-core kernel used by sbl_forward and sbl_backward for
+ * all later calls in this process: 0 = pairs of CTAs computing 256 x 256
+ * tiles with tcgen05 cta_group::2 (the default), 1 = one CTA per 128 x 256
+ * tile.  Results are identical (integer forward) or differ only in fp32
+ * summation order (backward).  Not a per-stream setting: do not change it
+ * while calls are being enqueued from other threads. */
+sbl_status sbl_set_gemm_variant(int variant);
+
 /* Synchronise `stream`, then return (and clear) the first error latched by a
  * kernel of this library on the current device since the previous check;
  * SBL_OK if none.  Also reports a pending CUDA error as SBL_ERR_CUDA. */

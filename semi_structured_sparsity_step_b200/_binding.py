@@ -23,6 +23,7 @@ SIGNATURES = {
     "sbl_status_string": (ctypes.c_char_p, [_c_int]),
     "sbl_version": (_c_int, []),
     "sbl_check": (_c_int, [_vp]),
+    "sbl_set_gemm_variant": (_c_int, [_c_int]),
     "sbl_mask_quant_workspace_bytes": (_c_size, [_c_int, _c_int]),
     "sbl_mask_quant": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
     "sbl_act_quant": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp]),
@@ -95,6 +96,10 @@ def sbl_status_string(status: int) -> str:
 
 def sbl_version() -> int:
     return load().sbl_version()
+
+
+def sbl_set_gemm_variant(variant: int) -> None:
+    _call("sbl_set_gemm_variant", int(variant))
 
 
 def sbl_check(stream=None) -> None:

@@ -308,6 +308,215 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------ CTA-pair kernel
+// Same product with a cluster of two CTAs per 256 x 256 tile (tcgen05
+// cta_group::2): CTA r of the pair stages rows [128 r, 128 r + 128) of the A
+// tile and rows [128 r, 128 r + 128) of the B tile (N half); the even CTA
+// issues tcgen05.mma with M = 256, which reads both CTAs' shared memory and
+// writes 128 accumulator rows into each CTA's TMEM.  Per SM this halves the
+// B bytes staged and read per MMA compared with a 128 x 256 tile on one SM.
+//   full[s]   (even CTA only): the even producer arms it with both CTAs' bytes;
+//             both producers' TMA loads complete on it.
+//   empty[s]  (both CTAs): freed by one multicast tcgen05.commit.
+//   tfull[b]  (both CTAs): accumulator buffer b ready (multicast commit).
+//   tempty[b] (even CTA only): 4 epilogue warps of each CTA arrive.
+template <bool kI8, bool kAMN, bool kBMN, int STAGES>
+struct Cfg2 {
+  static constexpr int BN = 256;                 // N of the pair's tile
+  static constexpr int BK = kI8 ? 128 : 64;      // elements per stage along K (128 bytes)
+  static constexpr int UK = kI8 ? 32 : 16;       // K per tcgen05.mma (32 bytes)
+  static constexpr int A_BYTES = 128 * 128;      // this CTA's 128 A rows
+  static constexpr int B_BYTES = 128 * 128;      // this CTA's 128 B rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_WARP_FLOATS = 32 * 33;
+  static constexpr int EPI_BYTES = 4 * EPI_WARP_FLOATS * 4;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr uint32_t IDESC = instr_desc(kI8, 256, BN, kAMN, kBMN);
+};
+
+template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmArgs args, const Sched sched) {
+  using C = Cfg2<kI8, kAMN, kBMN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* epi_tiles = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = pair::cluster_rank();
+  const bool leader = rank == 0;
+  const int pair_id = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int KB = (args.K + C::BK - 1) / C::BK;
+  const uint32_t peer_abort = pair::map_to(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    pair::tmem_alloc(tmem_slot, C::TMEM_COLS);
+    pair::tmem_relinquish();
+  }
+  tc_fence_before();
+  pair::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    pair::store_remote_u32(peer_abort, 1u);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int w = pair_id; w < sched.total && ok; w += n_pairs) {
+        int mb, nb, sp;
+        sched.item(w, mb, nb, sp);
+        const int kb0 = sp * args.kb_per_split;
+        const int kb1 = min(KB, kb0 + args.kb_per_split);
+        const int m0 = mb * 256 + 128 * static_cast<int>(rank);
+        const int n0 = nb * C::BN + 128 * static_cast<int>(rank);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t round = static_cast<uint32_t>(it / STAGES);
+          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, args.err)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE_BYTES);
+          const uint32_t fbar = pair::map_to(smem_u32(&full[s]), 0u);
+          uint8_t* sa = smem + s * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          const int kc = kb * C::BK;
+          if constexpr (!kAMN) {
+            pair::tma_load_2d(sa, &tmA, fbar, kc, m0);
+          } else {
+            pair::tma_load_2d(sa, &tmA, fbar, m0, kc);
+            pair::tma_load_2d(sa + C::BK * 128, &tmA, fbar, m0 + 64, kc);
+          }
+          if constexpr (!kBMN) {
+            pair::tma_load_2d(sb, &tmB, fbar, kc, n0);
+          } else {
+            pair::tma_load_2d(sb, &tmB, fbar, n0, kc);
+            pair::tma_load_2d(sb + C::BK * 128, &tmB, fbar, n0 + 64, kc);
+          }
+          ++it;
+        }
+      }
+      if (!ok && leader) {
+        for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i)
+          mbar_wait(&full[i % STAGES], static_cast<uint32_t>(i / STAGES) & 1u, nullptr, args.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      int it = 0, t = 0;
+      bool ok = true;
+      for (int w = pair_id; w < sched.total && ok; w += n_pairs, ++t) {
+        int mb, nb, sp;
+        sched.item(w, mb, nb, sp);
+        const int kb0 = sp * args.kb_per_split;
+        const int kb1 = min(KB, kb0 + args.kb_per_split);
+        const int b = t & 1;
+        if (!mbar_wait(&tempty[b], (static_cast<uint32_t>(t >> 1) & 1u) ^ 1u, abort_flag, args.err)) {
+          give_up();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * C::BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t round = static_cast<uint32_t>(it / STAGES);
+          if (!mbar_wait(&full[s], round & 1u, abort_flag, args.err)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::BK / C::UK; ++kk) {
+            const uint64_t adesc = kAMN ? smem_desc_sw128(sa + kk * C::UK * 128, C::BK * 128, 1024)
+                                        : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bdesc = kBMN ? smem_desc_sw128(sb + kk * C::UK * 128, C::BK * 128, 1024)
+                                        : smem_desc_sw128(sb + kk * 32, 16, 1024);
+            pair::umma<kI8>(d_tmem, adesc, bdesc, C::IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          pair::umma_commit_multicast(&empty[s], 0x3);
+          ++it;
+        }
+        pair::umma_commit_multicast(&tfull[b], 0x3);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    float* tile = epi_tiles + q * C::EPI_WARP_FLOATS;
+    int t = 0;
+    for (int w = pair_id; w < sched.total; w += n_pairs, ++t) {
+      int mb, nb, sp;
+      sched.item(w, mb, nb, sp);
+      const int b = t & 1;
+      if (!mbar_wait(&tfull[b], static_cast<uint32_t>(t >> 1) & 1u, abort_flag, args.err)) {
+        give_up();
+        break;
+      }
+      tc_fence_after();
+      if (*abort_flag) break;
+      const int row0 = mb * 256 + 128 * static_cast<int>(rank) + 32 * q;
+      const int row = row0 + lane;
+      float scale = 0.0f;
+      if constexpr (EPI == kEpiFwd) {
+        if (row < args.M) scale = __fmul_rn(*args.gamma, __fdiv_rn(args.amax[row], 127.0f));
+      } else if constexpr (EPI == kEpiDx) {
+        scale = *args.gamma;
+      }
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b * C::BN);
+#pragma unroll 1
+      for (int c = 0; c < C::BN / 32; ++c) {
+        const int col0 = nb * C::BN + 32 * c;
+        if (col0 >= args.N) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(32 * c), r);
+        tmem_ld_wait();
+        epilogue_chunk<EPI>(args, tile, row0, col0, lane, r, scale);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) pair::mbar_arrive_remote(pair::map_to(smem_u32(&tempty[b]), 0u));
+    }
+  }
+  tc_fence_before();
+  pair::cluster_sync();  // no MMA, copy or arrive of either CTA is still in flight
+  if (warp == 1) {
+    tc_fence_after();
+    pair::tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -360,8 +569,36 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
   return cudaGetLastError();
 }
 
+template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI>
+cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int splits, int num_sms,
+                     cudaStream_t stream) {
+  using C = Cfg2<kI8, kAMN, kBMN, STAGES>;
+  auto kern = tc_gemm_pair_kernel<kI8, kAMN, kBMN, STAGES, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  Sched sc;
+  sc.Mt = (a.M + 255) / 256;
+  sc.Nt = (a.N + C::BN - 1) / C::BN;
+  sc.splits = splits;
+  sc.total = sc.Mt * sc.Nt * splits;
+  int pairs = num_sms / 2;
+  if (pairs > sc.total) pairs = sc.total;
+  kern<<<2 * pairs, kThreads, C::SMEM_BYTES, stream>>>(ta, tb, a, sc);
+  return cudaGetLastError();
+}
+
 constexpr int kBN = 256;
 constexpr int kStages = 4;
+constexpr int kPairStages = 6;
+
+}  // namespace
+
+// Which tensor-core kernel the products use: 0 = CTA pairs (default),
+// 1 = one CTA per 128 x 256 tile.  Process-wide; set through
+// sbl_set_gemm_variant().
+int g_gemm_variant = 0;
+
+namespace {
 
 }  // namespace
 
@@ -375,9 +612,10 @@ cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_
       e = cudaMemsetAsync(acc, 0, sizeof(int32_t) * static_cast<size_t>(T) * d_out, stream);
     return e;
   }
+  const bool use_pair = g_gemm_variant == 0;
   CUtensorMap ta, tb;
   if (!make_tmap(&ta, Xq, false, d_in, T, d_in, 128, BM)) return cudaErrorInvalidValue;
-  if (!make_tmap(&tb, W_eff, false, d_in, d_out, d_in, 128, kBN)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tb, W_eff, false, d_in, d_out, d_in, 128, use_pair ? 128 : kBN)) return cudaErrorInvalidValue;
   GemmArgs a{};
   a.M = T;
   a.N = d_out;
@@ -389,12 +627,14 @@ cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_
   a.amax = amax;
   a.gamma = gamma;
   a.err = err;
+  if (use_pair) return run_pair<true, false, false, kPairStages, kEpiFwd>(ta, tb, a, 1, num_sms, stream);
   return run<true, false, false, kBN, kStages, kEpiFwd>(ta, tb, a, 1, num_sms, stream);
 }
 
 cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf16, const float* gamma, int T,
                             int d_in, int d_out, float* dX, float* dW, int accumulate_dW, cudaStream_t stream,
                             int num_sms, uint32_t* err) {
+  const bool use_pair = g_gemm_variant == 0;
   cudaError_t e = cudaSuccess;
   if (dX != nullptr && T > 0 && d_in > 0) {
     if (d_out == 0) {
@@ -413,7 +653,8 @@ cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf1
       a.ldo = d_in;
       a.gamma = gamma;
       a.err = err;
-      e = run<false, false, true, kBN, kStages, kEpiDx>(ta, tb, a, 1, num_sms, stream);
+      e = use_pair ? run_pair<false, false, true, kPairStages, kEpiDx>(ta, tb, a, 1, num_sms, stream)
+                   : run<false, false, true, kBN, kStages, kEpiDx>(ta, tb, a, 1, num_sms, stream);
     }
     if (e != cudaSuccess) return e;
   }
@@ -427,8 +668,9 @@ cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf1
     if (!make_tmap(&ta, dY, true, d_out, T, 2ull * d_out, 64, 64)) return cudaErrorInvalidValue;
     if (!make_tmap(&tb, X, true, d_in, T, 2ull * d_in, 64, 64)) return cudaErrorInvalidValue;
     const int KB = (T + 63) / 64;
-    const int tiles = ((d_in + kBN - 1) / kBN) * ((d_out + BM - 1) / BM);
-    int splits = num_sms / tiles;
+    const int tiles = use_pair ? ((d_in + 255) / 256) * ((d_out + 255) / 256)
+                               : ((d_in + kBN - 1) / kBN) * ((d_out + BM - 1) / BM);
+    int splits = (use_pair ? num_sms / 2 : num_sms) / tiles;
     if (splits < 1) splits = 1;
     if (splits > KB) splits = KB;
     const int kbps = (KB + splits - 1) / splits;
@@ -447,7 +689,8 @@ cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf1
       e = cudaMemsetAsync(dW, 0, sizeof(float) * static_cast<size_t>(d_out) * d_in, stream);
       if (e != cudaSuccess) return e;
     }
-    e = run<false, true, true, kBN, kStages, kEpiDw>(ta, tb, a, splits, num_sms, stream);
+    e = use_pair ? run_pair<false, true, true, kPairStages, kEpiDw>(ta, tb, a, splits, num_sms, stream)
+                 : run<false, true, true, kBN, kStages, kEpiDw>(ta, tb, a, splits, num_sms, stream);
   }
   return e;
 }

@@ -94,6 +94,12 @@ const char* sbl_status_string(int status) {
 
 int sbl_version(void) { return 100; }
 
+sbl_status sbl_set_gemm_variant(int variant) {
+  if (variant != 0 && variant != 1) return SBL_ERR_INVALID_ARG;
+  g_gemm_variant = variant;
+  return SBL_OK;
+}
+
 sbl_status sbl_check(void* stream) {
   DeviceInfo* d = nullptr;
   sbl_status st = current_device(&d);

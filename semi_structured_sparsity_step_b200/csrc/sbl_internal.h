@@ -29,6 +29,7 @@ cudaError_t launch_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* 
                              int num_sms);
 
 // ---- tensor-core GEMMs (gemm_tc.cu)
+extern int g_gemm_variant;
 cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
                            int d_in, int d_out, float* Y, int32_t* acc, cudaStream_t stream, int num_sms,
                            uint32_t* err);

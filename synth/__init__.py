@@ -115,17 +115,18 @@ def with_boundary_ties(w: torch.Tensor, N: int, M: int, seed: int = 0, tensor_id
     n_tie = max(1, int(round(frac * G)))
     chosen = torch.randperm(G, generator=g)[: n_tie + all_equal_groups]
     tie_groups, eq_groups = chosen[:n_tie], chosen[n_tie:]
-    for gi in tie_groups.tolist():
-        large = (2.0 + torch.rand(N - 1, generator=g)) * s
-        small = torch.rand(M - N - 1, generator=g) * s
-        tie = torch.full((2,), 1.5 * s)
-        mags = torch.cat([large, tie, small])
-        perm = torch.randperm(M, generator=g)
-        sign = torch.where(torch.rand(M, generator=g) < 0.5, -1.0, 1.0)
-        out[gi, perm] = mags * sign
-    for gi in eq_groups.tolist():
-        sign = torch.where(torch.rand(M, generator=g) < 0.5, -1.0, 1.0)
-        out[gi] = 1.5 * s * sign
+    large = (2.0 + torch.rand(n_tie, N - 1, generator=g)) * s
+    small = torch.rand(n_tie, M - N - 1, generator=g) * s
+    tie = torch.full((n_tie, 2), 1.5 * s)
+    mags = torch.cat([large, tie, small], dim=1)
+    perm = torch.argsort(torch.rand(n_tie, M, generator=g), dim=1)  # a random permutation per group
+    sign = torch.where(torch.rand(n_tie, M, generator=g) < 0.5, -1.0, 1.0)
+    rows = torch.empty(n_tie, M)
+    rows.scatter_(1, perm, mags * sign)
+    out[tie_groups] = rows
+    if all_equal_groups:
+        esign = torch.where(torch.rand(len(eq_groups), M, generator=g) < 0.5, -1.0, 1.0)
+        out[eq_groups] = 1.5 * s * esign
     # 1.5 s, 2 s .. 3 s are rounded to bf16 once here; equal inputs stay equal.
     return out.reshape(d_out, d_in).to(torch.bfloat16)
 
@@ -176,12 +177,15 @@ def layer_set(name: str) -> LayerSet:
 
     q/o: hidden x hidden, k/v: kv_dim x hidden, gate/up: intermediate x
     hidden, down: hidden x intermediate.  q, k and v read the attention input;
-    gate and up read the MLP input.
+    gate and up read the MLP input.  "qwen2.5-3b-up" is the up projection of
+    the 3B block alone (11008 x 2048).
     """
     shapes = {
         "qwen2.5-0.5b": (896, 4864, 128),
         "qwen2.5-3b": (2048, 11008, 256),
     }
+    if name == "qwen2.5-3b-up":
+        return LayerSet(name, 2048, 11008, 256, (Projection("up", 11008, 2048, "mlp_in"),))
     h, i, kv = shapes[name]
     projs = (
         Projection("q", h, h, "attn_in"),

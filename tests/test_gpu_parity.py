@@ -80,12 +80,20 @@ def _full_parity(lib, w, x, dy, N, M):
     return g, ref
 
 
+@pytest.fixture(params=[0, 1], ids=["pair", "single"])
+def variant(lib, request):
+    """Runs a test with each tensor-core kernel variant (CTA pairs, one CTA)."""
+    lib.sbl_set_gemm_variant(request.param)
+    yield request.param
+    lib.sbl_set_gemm_variant(0)
+
+
 def test_library_loads_on_gpu(lib):
     assert lib.sbl_version() >= 100
     lib.sbl_check()
 
 
-def test_single_layer_256_6of8_full_parity(lib):
+def test_single_layer_256_6of8_full_parity(lib, variant):
     """One 256 x 256 layer, 64 tokens, 6:8, W ~ N(0, 0.02), X, dY ~ N(0, 1)."""
     w = synth.normal_weight(256, 256, seed=0, tensor_id=0)
     x = synth.activations(64, 256, seed=0, tensor_id=100)
@@ -98,7 +106,7 @@ def test_single_layer_256_6of8_full_parity(lib):
     (1, 8, 16, 6, 8), (7, 136, 48, 2, 4), (129, 264, 272, 6, 8), (200, 392, 400, 4, 8),
     (130, 256, 1040, 3, 4), (333, 520, 144, 8, 8), (64, 8, 2064, 1, 8),
 ])
-def test_ragged_shapes(lib, T, d_out, d_in, N, M):
+def test_ragged_shapes(lib, variant, T, d_out, d_in, N, M):
     """Sizes that are not tile multiples (tiles are 128 x 256 x 128 bytes)."""
     w = synth.trimodal_weight(d_out, d_in, seed=3, tensor_id=T)
     x = synth.activations(T, d_in, seed=3, tensor_id=100 + T, outlier_frac=0.01)
@@ -138,7 +146,7 @@ def test_gamma_exact_on_extreme_magnitudes(lib):
     assert np.array_equal(L.W_eff.cpu().numpy(), weff)
 
 
-def test_dw_split_k_and_accumulate(lib):
+def test_dw_split_k_and_accumulate(lib, variant):
     """Small d_out (k/v-like) takes the split-K path with atomics; the
     accumulate flag adds into an existing gradient."""
     T, d_out, d_in = 1000, 128, 512
