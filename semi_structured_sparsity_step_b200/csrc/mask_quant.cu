@@ -51,6 +51,19 @@ __device__ __forceinline__ void gamma_add_bf16(uint32_t h, uint64_t& acc, unsign
   }
 }
 
+// Same split as gamma_add_bf16, with the in-window magnitude added to an fp64
+// partial sum (exact: see gamma_reduce_kernel).
+__device__ __forceinline__ void gamma_add_bf16_f64(uint32_t h, double& dacc, unsigned long long* sbucket) {
+  const uint32_t mag = h & 0x7FFFu;
+  if (mag - (static_cast<uint32_t>(kWinLo) << 7) < (32u << 7)) {
+    dacc += static_cast<double>(__uint_as_float(mag << 16));
+  } else {
+    const uint32_t e = mag >> 7;
+    const uint32_t m = (mag & 0x7Fu) | (e ? 0x80u : 0u);
+    if (m != 0u) atomicAdd(&sbucket[e ? e : 1u], static_cast<unsigned long long>(m));
+  }
+}
+
 // limbs (10 x 32 bit, little-endian) += v << shift, 0 <= shift < 256.
 __device__ void bigint_add_shifted(uint32_t* limbs, uint64_t v, int shift) {
   if (v == 0) return;
@@ -100,7 +113,7 @@ __device__ double bigint_to_double(const uint32_t* limbs) {
 
 // Largest bf16 magnitude pattern b (0 <= b < 0x7F80) with fp32(bf16(b) / den) <= 0.5.
 // fp32(|w| / den) is monotone in |w|, so W_q = 0 exactly when |w|'s pattern <= b.
-__device__ uint32_t zero_threshold_bits(float den) {
+__device__ uint32_t zero_threshold_bits_serial(float den) {
   uint32_t lo = 0u, hi = 0x7F80u;  // cond(lo) holds; cond(hi) fails (inf)
   while (hi - lo > 1u) {
     const uint32_t mid = (lo + hi) >> 1;
@@ -108,6 +121,30 @@ __device__ uint32_t zero_threshold_bits(float den) {
     if (__fdiv_rn(v, den) <= 0.5f) lo = mid; else hi = mid;
   }
   return lo;
+}
+
+// The same threshold found by one warp: the boundary lies within a bf16 ulp
+// of den / 2, so the 32 lanes test the 32 patterns around it with the IEEE
+// divide at once and the boundary is the last lane that passes.  If the
+// window does not bracket the boundary (not expected), lane 0 falls back to
+// the serial search.  Must be called by all 32 lanes; returns in every lane.
+__device__ uint32_t zero_threshold_bits_warp(float den) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t centre = __float_as_uint(__fmul_rn(den, 0.5f)) >> 16;  // truncated to bf16
+  const int base = static_cast<int>(centre) - 16;
+  const int cand = base + static_cast<int>(lane);
+  bool ok = false;
+  if (cand >= 0 && cand < 0x7F80) ok = __fdiv_rn(__uint_as_float(static_cast<uint32_t>(cand) << 16), den) <= 0.5f;
+  const uint32_t pass = __ballot_sync(0xFFFFFFFFu, ok);
+  uint32_t thr;
+  const bool bracketed = (pass & 1u) && !(pass >> 31) && ((pass & (pass + 1u)) == 0u);  // a prefix 0..k, k < 31
+  if (bracketed) {
+    thr = static_cast<uint32_t>(base + (31 - __clz(pass)));
+  } else {
+    thr = lane == 0 ? zero_threshold_bits_serial(den) : 0u;
+    thr = __shfl_sync(0xFFFFFFFFu, thr, 0);
+  }
+  return thr;
 }
 
 __global__ void __launch_bounds__(kGammaThreads) gamma_reduce_kernel(const uint4* __restrict__ W, size_t n_vec,
@@ -119,9 +156,33 @@ __global__ void __launch_bounds__(kGammaThreads) gamma_reduce_kernel(const uint4
   sbucket[threadIdx.x] = 0ull;
   __syncthreads();
 
+  // In-window magnitudes (|w| in [2^-31, 2), bf16 pattern in [0x3000, 0x4000))
+  // are added as fp64: each is a multiple of 2^-38 below 2, so a sum of up to
+  // 512 of them stays below 2^10 and needs at most 48 significant bits --
+  // every fp64 addition is exact.  The partial sum is moved into the uint64
+  // `acc` (units of 2^-38) every 512 elements.
   uint64_t acc = 0;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_vec;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  while (i + 3 * stride < n_vec) {
+    double dacc = 0.0;
+    for (int rep = 0; rep < 16 && i + 3 * stride < n_vec; ++rep, i += 4 * stride) {  // 16 x 32 elements
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldg(W + i + u * stride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          gamma_add_bf16_f64(w4[k] & 0xFFFFu, dacc, sbucket);
+          gamma_add_bf16_f64(w4[k] >> 16, dacc, sbucket);
+        }
+      }
+    }
+    acc += static_cast<uint64_t>(scalbn(dacc, 38));
+  }
+  for (; i < n_vec; i += stride) {
     const uint4 v = __ldg(W + i);
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -147,100 +208,143 @@ __global__ void __launch_bounds__(kGammaThreads) gamma_reduce_kernel(const uint4
   if (!s_last) return;
   __threadfence();
 
-  // Last block: 128-bit sum of the per-block window sums.
-  __shared__ uint64_t s_lo[kGammaThreads], s_hi[kGammaThreads];
+  // Last block: 128-bit sum of the per-block window sums, one lane per
+  // partial, then a shuffle tree; carries are tracked in the high word.
+  __shared__ uint64_t s_lo[kGammaThreads / 32], s_hi[kGammaThreads / 32];
+  __shared__ uint32_t s_occ[256 / 32];
+  __shared__ float s_gamma;
   uint64_t lo = 0, hi = 0;
   for (unsigned b = threadIdx.x; b < gridDim.x; b += blockDim.x) {
     const uint64_t p = __ldcg(&ws->block_window[b]);
     lo += p;
     hi += (lo < p) ? 1u : 0u;
   }
-  s_lo[threadIdx.x] = lo;
-  s_hi[threadIdx.x] = hi;
-  sbucket[threadIdx.x] = __ldcg(&ws->bucket[threadIdx.x]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t olo = __shfl_xor_sync(0xFFFFFFFFu, lo, o);
+    const uint64_t ohi = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
+    lo += olo;
+    hi += ohi + ((lo < olo) ? 1u : 0u);
+  }
+  const uint64_t bucket = __ldcg(&ws->bucket[threadIdx.x]);
+  sbucket[threadIdx.x] = bucket;
+  const uint32_t occ = __ballot_sync(0xFFFFFFFFu, bucket != 0ull);
+  if ((threadIdx.x & 31) == 0) {
+    s_lo[threadIdx.x >> 5] = lo;
+    s_hi[threadIdx.x >> 5] = hi;
+    s_occ[threadIdx.x >> 5] = occ;
+  }
   __syncthreads();
-  if (threadIdx.x != 0) return;
-  lo = 0;
-  hi = 0;
-  for (int t = 0; t < kGammaThreads; ++t) {
-    lo += s_lo[t];
-    hi += s_hi[t] + ((lo < s_lo[t]) ? 1u : 0u);
-  }
-  uint32_t limbs[kGammaLimbs];
-#pragma unroll
-  for (int i = 0; i < kGammaLimbs; ++i) limbs[i] = 0u;
-  // value = m * 2^(ee-134) = m * 2^(ee-1) units of 2^-133; window sums carry 2^(96-1).
-  bigint_add_shifted(limbs, lo, kWinLo - 1);
-  bigint_add_shifted(limbs, hi, kWinLo - 1 + 64);
-  for (int ee = 1; ee < 256; ++ee) bigint_add_shifted(limbs, sbucket[ee], ee - 1);
-  const double total = bigint_to_double(limbs);
-  const double mean = __ddiv_rn(total, static_cast<double>(n_elems));
-  const float gamma = __double2float_rn(mean);
-  *gamma_out = gamma;
-  ws->zero_threshold = zero_threshold_bits(__fadd_rn(gamma, 1e-5f));
-}
-
-
-template <int M>
-__device__ __forceinline__ void rank_keep(const uint32_t (&mag)[8], int N, uint32_t& keep_bits) {
-  // key = magnitude, then lower position first; all keys in a group differ.
-  keep_bits = 0u;
-#pragma unroll
-  for (int g = 0; g < 8 / M; ++g) {
-    uint32_t key[M];
-    int rank[M];
-#pragma unroll
-    for (int j = 0; j < M; ++j) {
-      key[j] = (mag[g * M + j] << 3) | static_cast<uint32_t>(M - 1 - j);
-      rank[j] = 0;
-    }
-#pragma unroll
-    for (int i = 0; i < M; ++i) {
-#pragma unroll
-      for (int j = i + 1; j < M; ++j) {
-        const int gt = key[i] > key[j];
-        rank[j] += gt;
-        rank[i] += 1 - gt;
+  if (threadIdx.x < 32) {
+    if (threadIdx.x == 0) {
+      lo = 0;
+      hi = 0;
+      for (int w = 0; w < kGammaThreads / 32; ++w) {
+        lo += s_lo[w];
+        hi += s_hi[w] + ((lo < s_lo[w]) ? 1u : 0u);
       }
-    }
+      uint32_t limbs[kGammaLimbs];
 #pragma unroll
-    for (int j = 0; j < M; ++j) keep_bits |= (rank[j] < N ? 1u : 0u) << (g * M + j);
+      for (int i = 0; i < kGammaLimbs; ++i) limbs[i] = 0u;
+      // value = m * 2^(ee-134) = m * 2^(ee-1) units of 2^-133; window sums carry 2^(96-1).
+      bigint_add_shifted(limbs, lo, kWinLo - 1);
+      bigint_add_shifted(limbs, hi, kWinLo - 1 + 64);
+      for (int w = 0; w < 256 / 32; ++w) {
+        uint32_t m = s_occ[w];
+        while (m != 0u) {  // only the occupied exponent buckets
+          const int ee = 32 * w + (__ffs(m) - 1);
+          m &= m - 1u;
+          if (ee >= 1) bigint_add_shifted(limbs, sbucket[ee], ee - 1);
+        }
+      }
+      const double total = bigint_to_double(limbs);
+      const double mean = __ddiv_rn(total, static_cast<double>(n_elems));
+      s_gamma = __double2float_rn(mean);
+      *gamma_out = s_gamma;
+    }
+    __syncwarp();
+    const uint32_t thr = zero_threshold_bits_warp(__fadd_rn(s_gamma, 1e-5f));
+    if (threadIdx.x == 0) ws->zero_threshold = thr;
   }
 }
 
-template <int M>
-__global__ void __launch_bounds__(256) ternary_mask_kernel(const uint4* __restrict__ W, size_t n_vec, int N,
+
+// Keep flags of one group of M positions (bit j = position j).  Each
+// position gets the key (|w| pattern << 3) | (M-1-j): all keys of a group
+// differ, and a larger key means "kept first" (larger magnitude, then lower
+// index).  The group keeps its N largest keys.  Whichever side is smaller is
+// selected by repeated minimum/maximum reductions: with d = M - N <= N the d
+// smallest keys are dropped, otherwise the N largest are kept.  Subtracting
+// (last + 1) with unsigned wrap-around moves the keys already taken to the
+// top (for the minimum) so each round is one sub and one min per key.
+template <int M, int N>
+__device__ __forceinline__ uint32_t keep_group(const uint32_t (&key)[M]) {
+  constexpr int d = M - N;
+  if constexpr (d == 0) return (1u << M) - 1u;
+  if constexpr (d <= N) {
+    uint32_t dropped = 0u, last = 0u;
+#pragma unroll
+    for (int r = 0; r < d; ++r) {
+      const uint32_t off = r == 0 ? 0u : last + 1u;
+      uint32_t mn = 0xFFFFFFFFu;
+#pragma unroll
+      for (int j = 0; j < M; ++j) mn = min(mn, key[j] - off);
+      last = mn + off;
+      dropped |= 1u << (M - 1 - static_cast<int>(last & 7u));
+    }
+    return ((1u << M) - 1u) & ~dropped;
+  }
+  uint32_t kept = 0u, last = 0xFFFFFFFFu;
+#pragma unroll
+  for (int r = 0; r < N; ++r) {
+    uint32_t mx = 0u;
+#pragma unroll
+    for (int j = 0; j < M; ++j) mx = max(mx, key[j] < last ? key[j] : 0u);
+    last = mx;
+    kept |= 1u << (M - 1 - static_cast<int>(mx & 7u));
+  }
+  return kept;
+}
+
+template <int M, int N>
+__global__ void __launch_bounds__(256) ternary_mask_kernel(const uint4* __restrict__ W, size_t n_vec,
                                                            const GammaWorkspace* __restrict__ ws,
                                                            uint2* __restrict__ w_eff,
                                                            uint4* __restrict__ w_eff_bf16,
                                                            uint8_t* __restrict__ mask_bits) {
   const uint32_t thr = ws->zero_threshold;
+  const uint32_t thr2 = thr | (thr << 16);
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_vec;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const uint4 v = __ldg(W + i);
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-    uint32_t h[8], mag[8];
+    // ---- N:M mask from the 15-bit magnitudes
+    uint32_t keep = 0u;
+#pragma unroll
+    for (int g = 0; g < 8 / M; ++g) {
+      uint32_t key[M];
+#pragma unroll
+      for (int j = 0; j < M; ++j) {
+        const int pos = g * M + j;
+        const uint32_t h = (w4[pos >> 1] >> (16 * (pos & 1))) & 0x7FFFu;
+        key[j] = (h << 3) | static_cast<uint32_t>(M - 1 - j);
+      }
+      keep |= keep_group<M, N>(key) << (g * M);
+    }
+    // ---- ternary codes, two bf16 per 32-bit word
+    uint32_t qb[4], q16[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      h[2 * k] = w4[k] & 0xFFFFu;
-      h[2 * k + 1] = w4[k] >> 16;
+      const uint32_t mag = w4[k] & 0x7FFF7FFFu;
+      const uint32_t gt = __vcmpgtu2(mag, thr2);                           // 0xFFFF where |w| maps to +-1
+      const uint32_t kb = (keep >> (2 * k)) & 3u;
+      const uint32_t kh = ((kb & 1u) | ((kb & 2u) << 15)) * 0xFFFFu;        // keep flags as 16-bit lanes
+      const uint32_t nz = gt & kh;
+      const uint32_t neg = ((w4[k] >> 15) & 0x00010001u) * 0xFFFFu;         // sign as 16-bit lanes
+      qb[k] = nz & (0x3F803F80u | (w4[k] & 0x80008000u));                  // +-1.0 in bf16
+      q16[k] = nz & (0x00010001u | neg);                                   // +-1 in int16 lanes
     }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) mag[k] = h[k] & 0x7FFFu;
-    uint32_t keep;
-    rank_keep<M>(mag, N, keep);
-    uint32_t q8[2] = {0u, 0u};
-    uint32_t qb[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const bool nz = ((keep >> k) & 1u) && (mag[k] > thr);
-      const bool neg = (h[k] >> 15) != 0u;
-      const uint32_t byte = nz ? (neg ? 0xFFu : 0x01u) : 0u;
-      const uint32_t bf = nz ? (neg ? 0xBF80u : 0x3F80u) : 0u;
-      q8[k >> 2] |= byte << (8 * (k & 3));
-      qb[k >> 1] |= bf << (16 * (k & 1));
-    }
-    w_eff[i] = make_uint2(q8[0], q8[1]);
+    w_eff[i] = make_uint2(__byte_perm(q16[0], q16[1], 0x6420), __byte_perm(q16[2], q16[3], 0x6420));
     if (w_eff_bf16 != nullptr) w_eff_bf16[i] = make_uint4(qb[0], qb[1], qb[2], qb[3]);
     if (mask_bits != nullptr) mask_bits[i] = static_cast<uint8_t>(keep);
   }
@@ -266,18 +370,35 @@ cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   size_t qblocks = (n_vec + 255) / 256;
-  const size_t qmax = static_cast<size_t>(num_sms) * 16;
+  const size_t qmax = static_cast<size_t>(num_sms) * 8;
   if (qblocks > qmax) qblocks = qmax;
   if (qblocks < 1) qblocks = 1;
+  const unsigned qb = static_cast<unsigned>(qblocks);
+  const uint4* w4 = static_cast<const uint4*>(W);
+  uint2* we = reinterpret_cast<uint2*>(W_eff);
+  uint4* wb = static_cast<uint4*>(W_eff_bf16);
+#define SBL_TERNARY(MM, NN) \
+  ternary_mask_kernel<MM, NN><<<qb, 256, 0, stream>>>(w4, n_vec, ws, we, wb, mask_bits)
   if (M == 8) {
-    ternary_mask_kernel<8><<<static_cast<unsigned>(qblocks), 256, 0, stream>>>(
-        static_cast<const uint4*>(W), n_vec, N, ws, reinterpret_cast<uint2*>(W_eff),
-        static_cast<uint4*>(W_eff_bf16), mask_bits);
+    switch (N) {
+      case 1: SBL_TERNARY(8, 1); break;
+      case 2: SBL_TERNARY(8, 2); break;
+      case 3: SBL_TERNARY(8, 3); break;
+      case 4: SBL_TERNARY(8, 4); break;
+      case 5: SBL_TERNARY(8, 5); break;
+      case 6: SBL_TERNARY(8, 6); break;
+      case 7: SBL_TERNARY(8, 7); break;
+      default: SBL_TERNARY(8, 8); break;
+    }
   } else {
-    ternary_mask_kernel<4><<<static_cast<unsigned>(qblocks), 256, 0, stream>>>(
-        static_cast<const uint4*>(W), n_vec, N, ws, reinterpret_cast<uint2*>(W_eff),
-        static_cast<uint4*>(W_eff_bf16), mask_bits);
+    switch (N) {
+      case 1: SBL_TERNARY(4, 1); break;
+      case 2: SBL_TERNARY(4, 2); break;
+      case 3: SBL_TERNARY(4, 3); break;
+      default: SBL_TERNARY(4, 4); break;
+    }
   }
+#undef SBL_TERNARY
   return cudaGetLastError();
 }
 
