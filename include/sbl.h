@@ -108,6 +108,32 @@ sbl_status sbl_mask_quant(const void* W, int d_out, int d_in, int N, int M,
                           void* stream);
 
 /* ------------------------------------------------------------------------
+ * sbl_mask_quant without a caller-supplied workspace.  The paper has no
+ * counterpart for this call: it exists for callers that cannot allocate
+ * device memory when the weight step runs, such as processes that reserve
+ * their whole device-memory budget at start-up and forbid any later
+ * cudaMalloc, or host frameworks whose plugin interface passes only the
+ * input and output buffers.  It computes exactly what sbl_mask_quant
+ * computes (same arguments, minus the workspace) and allocates nothing: the
+ * scratch is a fixed array of sbl_mask_quant_noalloc_scratch_bytes() bytes
+ * (7040) in the library's static device memory, which every device that
+ * loads the library holds until the process exits.
+ *   - Size limit: W may have at most 2^32 - 1 elements (d_out * d_in);
+ *     larger W returns SBL_ERR_SHAPE without launching anything.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (once per device, with that device current) and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the one scratch array.  Each call clears
+ *     the part that must start at zero, but calls that overlap on the GPU
+ *     (different streams, or different host threads without ordering) race
+ *     on it and give wrong results: order them on one stream.
+ * ---------------------------------------------------------------------- */
+size_t sbl_mask_quant_noalloc_scratch_bytes(void);
+sbl_status sbl_mask_quant_noalloc(const void* W, int d_out, int d_in, int N, int M,
+                                  int8_t* W_eff, void* W_eff_bf16, uint8_t* mask_bits,
+                                  float* gamma, void* stream);
+
+/* ------------------------------------------------------------------------
  * Per-token absmax int8 activation quantiser.
  * [summary] 前置知识 (activations absmax-quantised to 8-bit integers) and
  * Algorithm 1 step (3).

@@ -26,6 +26,8 @@ SIGNATURES = {
     "sbl_set_gemm_variant": (_c_int, [_c_int]),
     "sbl_mask_quant_workspace_bytes": (_c_size, [_c_int, _c_int]),
     "sbl_mask_quant": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
+    "sbl_mask_quant_noalloc_scratch_bytes": (_c_size, []),
+    "sbl_mask_quant_noalloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp]),
     "sbl_act_quant": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_forward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_backward_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
@@ -114,6 +116,19 @@ def sbl_mask_quant(W, d_out, d_in, N, M, W_eff, W_eff_bf16, mask_bits, gamma, wo
                    stream=None) -> None:
     _call("sbl_mask_quant", _ptr(W), d_out, d_in, N, M, _ptr(W_eff), _ptr(W_eff_bf16), _ptr(mask_bits),
           _ptr(gamma), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def sbl_mask_quant_noalloc_scratch_bytes() -> int:
+    return load().sbl_mask_quant_noalloc_scratch_bytes()
+
+
+def sbl_mask_quant_noalloc(W, d_out, d_in, N, M, W_eff, W_eff_bf16, mask_bits, gamma, stream=None) -> None:
+    """sbl_mask_quant for callers that cannot allocate device memory when
+    the weight step runs: the scratch is a fixed array in the library's
+    static device memory (see include/sbl.h for the size limit and for why
+    calls must be ordered on one stream)."""
+    _call("sbl_mask_quant_noalloc", _ptr(W), d_out, d_in, N, M, _ptr(W_eff), _ptr(W_eff_bf16), _ptr(mask_bits),
+          _ptr(gamma), _stream(stream))
 
 
 def sbl_act_quant(X, T, d_in, Xq, amax, stream=None) -> None:

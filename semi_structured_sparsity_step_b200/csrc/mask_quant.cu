@@ -30,7 +30,9 @@
 //      (lower index wins), using pairwise compares in registers.
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <mutex>
 
+#include "../../include/sbl.h"
 #include "sbl_device.cuh"
 #include "sbl_internal.h"
 
@@ -403,3 +405,73 @@ cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, 
 }
 
 }  // namespace sbl
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of sbl_mask_quant.
+//
+// Some callers cannot allocate device memory at the point where they run
+// the weight step: processes that reserve their whole device-memory budget
+// at start-up and forbid any later cudaMalloc, and host frameworks whose
+// plugin interface hands over only the input and output buffers, with no
+// workspace.  For them the scratch of the gamma pass (exponent buckets, the
+// finished-blocks ticket and one partial sum per block) lives in the fixed
+// array below, part of the library's own static device memory: every device
+// that loads the library holds these bytes until the process exits.
+namespace {
+
+static __device__ __align__(256) unsigned char g_mask_quant_scratch[sizeof(sbl::GammaWorkspace)];
+
+constexpr int kNoAllocMaxDevices = 64;
+void* g_scratch_ptr[kNoAllocMaxDevices] = {};
+int g_scratch_sms[kNoAllocMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device with that device current, and cached.
+sbl_status scratch_for_current_device(void** ptr, int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SBL_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return SBL_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SBL_ERR_CUDA;
+    if (major != 10 || minor != 0) return SBL_ERR_UNSUPPORTED;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_mask_quant_scratch) != cudaSuccess || p == nullptr) return SBL_ERR_CUDA;
+    g_scratch_sms[dev] = sms;
+    g_scratch_ptr[dev] = p;
+  }
+  *ptr = g_scratch_ptr[dev];
+  *num_sms = g_scratch_sms[dev];
+  return SBL_OK;
+}
+
+}  // namespace
+
+extern "C" size_t sbl_mask_quant_noalloc_scratch_bytes(void) { return sizeof(sbl::GammaWorkspace); }
+
+extern "C" sbl_status sbl_mask_quant_noalloc(const void* W, int d_out, int d_in, int N, int M, int8_t* W_eff,
+                                             void* W_eff_bf16, uint8_t* mask_bits, float* gamma, void* stream) {
+  if (!(M == 4 || M == 8) || N < 1 || N > M) return SBL_ERR_INVALID_ARG;
+  if (W == nullptr || W_eff == nullptr || gamma == nullptr) return SBL_ERR_INVALID_ARG;
+  if (d_out <= 0 || d_in <= 0 || d_in % 16 != 0 || d_out % 8 != 0 || d_in % M != 0) return SBL_ERR_SHAPE;
+  // The fixed scratch serves any W up to 2^32 - 1 elements; larger W is refused.
+  if (static_cast<unsigned long long>(d_out) * static_cast<unsigned long long>(d_in) >= (1ull << 32))
+    return SBL_ERR_SHAPE;
+  auto misaligned = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) != 0; };
+  if (misaligned(W) || misaligned(W_eff) || misaligned(W_eff_bf16) || misaligned(mask_bits) ||
+      (reinterpret_cast<uintptr_t>(gamma) & 3u) != 0)
+    return SBL_ERR_ALIGN;
+  void* scratch = nullptr;
+  int num_sms = 0;
+  const sbl_status st = scratch_for_current_device(&scratch, &num_sms);
+  if (st != SBL_OK) return st;
+  const cudaError_t e = sbl::launch_mask_quant(W, d_out, d_in, N, M, W_eff, W_eff_bf16, mask_bits, gamma, scratch,
+                                               static_cast<cudaStream_t>(stream), num_sms);
+  return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
+}
