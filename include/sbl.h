@@ -206,6 +206,23 @@ sbl_status sbl_gemv_packed(const int8_t* Xq, const float* amax, int batch,
                            const uint8_t* packed, const float* gamma, int d_in,
                            int d_out, int N, int M, float* Y, void* stream);
 
+/* Several decode GEMVs in one launch (e.g. the projections of a layer, or of
+ * several layers): problem i is exactly sbl_gemv_packed on its own buffers.
+ * Same citation as sbl_gemv_packed.
+ *   problems  HOST array of `count` descriptors (read before the call
+ *             returns; the pointers inside are device pointers).
+ *   batch     tokens (1..16), N:M shared by all problems. */
+typedef struct {
+  const uint8_t* packed; /* sbl_pack output of a [d_out, d_in] weight */
+  const int8_t* Xq;      /* [batch, d_in] int8 activations            */
+  const float* amax;     /* [batch] per-token absmax (sbl_act_quant)  */
+  const float* gamma;    /* 1 float, the weight's absmean scale       */
+  float* Y;              /* [batch, d_out] float out                  */
+  int d_in, d_out;
+} sbl_gemv_problem;
+sbl_status sbl_gemv_packed_group(const sbl_gemv_problem* problems, int count, int batch,
+                                 int N, int M, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

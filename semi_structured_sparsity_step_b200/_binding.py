@@ -18,6 +18,12 @@ _c_int = ctypes.c_int
 _c_size = ctypes.c_size_t
 _vp = ctypes.c_void_p
 
+class GemvProblem(ctypes.Structure):
+    """sbl_gemv_problem: one decode GEMV of a group (device pointers)."""
+    _fields_ = [("packed", _vp), ("Xq", _vp), ("amax", _vp), ("gamma", _vp), ("Y", _vp),
+                ("d_in", _c_int), ("d_out", _c_int)]
+
+
 # name -> (restype, argtypes)
 SIGNATURES = {
     "sbl_status_string": (ctypes.c_char_p, [_c_int]),
@@ -35,6 +41,7 @@ SIGNATURES = {
     "sbl_packed_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "sbl_pack": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
     "sbl_gemv_packed": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
+    "sbl_gemv_packed_group": (_c_int, [ctypes.POINTER(GemvProblem), _c_int, _c_int, _c_int, _c_int, _vp]),
 }
 
 STATUS = {
@@ -161,3 +168,11 @@ def sbl_pack(W_eff, d_out, d_in, N, M, packed, packed_bytes, stream=None) -> Non
 def sbl_gemv_packed(Xq, amax, batch, packed, gamma, d_in, d_out, N, M, Y, stream=None) -> None:
     _call("sbl_gemv_packed", _ptr(Xq), _ptr(amax), batch, _ptr(packed), _ptr(gamma), d_in, d_out, N, M, _ptr(Y),
           _stream(stream))
+
+
+def sbl_gemv_packed_group(problems, batch, N, M, stream=None) -> None:
+    """problems: sequence of (packed, Xq, amax, gamma, Y, d_in, d_out)."""
+    arr = (GemvProblem * len(problems))()
+    for i, (pk, xq, am, gm, y, d_in, d_out) in enumerate(problems):
+        arr[i] = GemvProblem(_ptr(pk), _ptr(xq), _ptr(am), _ptr(gm), _ptr(y), d_in, d_out)
+    _call("sbl_gemv_packed_group", arr, len(problems), batch, N, M, _stream(stream))

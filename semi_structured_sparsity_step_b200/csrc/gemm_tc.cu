@@ -552,6 +552,23 @@ bool make_tmap(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint
   return r == CUDA_SUCCESS;
 }
 
+}  // namespace
+
+bool make_tmap_u32(CUtensorMap* m, const void* base, unsigned long long inner, unsigned long long rows,
+                   unsigned long long row_bytes, unsigned box_inner, unsigned box_rows) {
+  EncodeTiledFn enc = encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
 template <bool kI8, bool kAMN, bool kBMN, int BN, int STAGES, int EPI>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int splits, int num_sms,
                 cudaStream_t stream) {

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <vector>
 
 #include "../../include/sbl.h"
 #include "sbl_device.cuh"
@@ -232,7 +233,32 @@ sbl_status sbl_gemv_packed(const int8_t* Xq, const float* amax, int batch, const
   DeviceInfo* d = nullptr;
   if ((st = current_device(&d)) != SBL_OK) return st;
   return from_cuda(launch_gemv_packed(Xq, amax, batch, packed, gamma, d_in, d_out, N, M, Y,
-                                      static_cast<cudaStream_t>(stream), d->num_sms));
+                                      static_cast<cudaStream_t>(stream), d->num_sms, d->err));
+}
+
+sbl_status sbl_gemv_packed_group(const sbl_gemv_problem* problems, int count, int batch, int N, int M,
+                                 void* stream) {
+  sbl_status st = check_nm(N, M);
+  if (st != SBL_OK) return st;
+  if (count < 0 || batch < 0 || batch > 16) return SBL_ERR_SHAPE;
+  if (count == 0 || batch == 0) return SBL_OK;
+  if (problems == nullptr) return SBL_ERR_INVALID_ARG;
+  std::vector<GemvProblemDev> dev(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    const sbl_gemv_problem& p = problems[i];
+    if ((st = check_dims(p.d_in, p.d_out)) != SBL_OK) return st;
+    if (p.d_in % M != 0 || p.d_in == 0) return SBL_ERR_SHAPE;
+    if (p.Xq == nullptr || p.amax == nullptr || p.packed == nullptr || p.gamma == nullptr || p.Y == nullptr)
+      return SBL_ERR_INVALID_ARG;
+    if (!aligned16(p.Xq) || !aligned16(p.amax) || !aligned16(p.packed) || !aligned16(p.Y) ||
+        (reinterpret_cast<uintptr_t>(p.gamma) & 3u) != 0)
+      return SBL_ERR_ALIGN;
+    dev[i] = GemvProblemDev{p.packed, p.Xq, p.amax, p.gamma, p.Y, p.d_in, p.d_out, 0, 0};
+  }
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  return from_cuda(launch_gemv_group(dev.data(), count, batch, N, M, static_cast<cudaStream_t>(stream), d->num_sms,
+                                     d->err));
 }
 
 }  // extern "C"

@@ -2,6 +2,7 @@
 // (launchers called by the C ABI in sbl_api.cu).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -29,6 +30,10 @@ cudaError_t launch_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* 
                              int num_sms);
 
 // ---- tensor-core GEMMs (gemm_tc.cu)
+// 2-D tensor map of a row-major [rows, inner] uint32 matrix (row stride in
+// bytes), box [box_rows, box_inner], no swizzle; out-of-range elements read 0.
+bool make_tmap_u32(CUtensorMap* m, const void* base, unsigned long long inner, unsigned long long rows,
+                   unsigned long long row_bytes, unsigned box_inner, unsigned box_rows);
 extern int g_gemm_variant;
 cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
                            int d_in, int d_out, float* Y, int32_t* acc, cudaStream_t stream, int num_sms,
@@ -42,8 +47,19 @@ size_t packed_codes_row_bytes(int d_in, int N, int M);
 size_t packed_index_row_bytes(int d_in, int M);
 cudaError_t launch_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M, uint8_t* packed,
                         cudaStream_t stream, uint32_t* err);
+struct GemvProblemDev {
+  const uint8_t* packed;
+  const int8_t* Xq;
+  const float* amax;
+  const float* gamma;
+  float* Y;
+  int d_in, d_out;
+  size_t crow, irow;  // filled in by the launcher
+};
+cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
+                              cudaStream_t stream, int num_sms, uint32_t* err);
 cudaError_t launch_gemv_packed(const int8_t* Xq, const float* amax, int batch, const uint8_t* packed,
                                const float* gamma, int d_in, int d_out, int N, int M, float* Y,
-                               cudaStream_t stream, int num_sms);
+                               cudaStream_t stream, int num_sms, uint32_t* err);
 
 }  // namespace sbl

@@ -249,3 +249,27 @@ def test_gamma_exact_on_log_uniform_magnitudes(lib):
         weff, gamma, _ = oracle.effective_weight(synth.bits(w), N, M)
         assert L.gamma.item() == float(gamma)
         assert np.array_equal(L.W_eff.cpu().numpy(), weff)
+
+
+def test_gemv_group_matches_single_calls(lib):
+    """One grouped launch over projections of different shapes equals the
+    per-projection results (and the oracle)."""
+    shapes = [(264, 2048), (8, 896), (520, 11008), (136, 4864)]
+    probs, refs = [], []
+    batch = 5
+    for i, (d_out, d_in) in enumerate(shapes):
+        w = synth.trimodal_weight(d_out, d_in, seed=30, tensor_id=i)
+        weff, gamma, _ = oracle.effective_weight(synth.bits(w), 6, 8)
+        x = synth.activations(batch, d_in, seed=30, tensor_id=100 + i)
+        xq, amax = oracle.act_quant(synth.bits(x))
+        nbytes = lib.sbl_packed_bytes(d_out, d_in, 6, 8)
+        packed = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        lib.sbl_pack(torch.from_numpy(weff).cuda(), d_out, d_in, 6, 8, packed, nbytes)
+        Y = torch.empty(batch, d_out, dtype=torch.float32, device="cuda")
+        g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+        probs.append((packed, torch.from_numpy(xq).cuda(), torch.from_numpy(amax).cuda(), g, Y, d_in, d_out))
+        refs.append(oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax))
+    lib.sbl_gemv_packed_group(probs, batch, 6, 8)
+    lib.sbl_check()
+    for (_, _, _, _, Y, _, _), ref in zip(probs, refs):
+        assert np.array_equal(Y.cpu().numpy(), ref)
