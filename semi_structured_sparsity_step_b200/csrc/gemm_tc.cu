@@ -68,17 +68,24 @@ struct Cfg {
   static constexpr uint32_t IDESC = instr_desc(kI8, BM, BN, kAMN, kBMN);
 };
 
-// Work item -> (m block, n block, k split).  n varies fastest, so the CTAs
-// that run at the same time share the weight-side (B) tiles and each A row
-// block is fetched from HBM once.
+// Work item -> (m block, n block, k split).  Items are ordered in strips of
+// GM consecutive m blocks: inside a strip m varies fastest, then n; k splits
+// are outermost.  GM = 1 is plain n-fastest order (the concurrent tiles share
+// the B tiles and each A row block is read once); GM = Mt makes all m blocks
+// of an n block run together so a streamed B operand is read once.  The
+// host picks GM from the operands' sizes.
 struct Sched {
-  int Mt, Nt, splits, total;
+  int Mt, Nt, splits, total, GM;
   __device__ __forceinline__ void item(int w, int& mb, int& nb, int& sp) const {
     const int per = Mt * Nt;
     sp = w / per;
-    const int r = w - sp * per;
-    mb = r / Nt;
-    nb = r - mb * Nt;
+    int r = w - sp * per;
+    const int strip_items = GM * Nt;
+    const int strip = r / strip_items;
+    r -= strip * strip_items;
+    const int gm = min(GM, Mt - strip * GM);  // the last strip may be narrower
+    nb = r / gm;
+    mb = strip * GM + (r - nb * gm);
   }
 };
 
@@ -581,14 +588,41 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
   sc.Nt = (a.N + BN - 1) / BN;
   sc.splits = splits;
   sc.total = sc.Mt * sc.Nt * splits;
+  sc.GM = 1;
   const int grid = sc.total < num_sms ? sc.total : num_sms;
   kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(ta, tb, a, sc);
   return cudaGetLastError();
 }
 
+// Strip height (m blocks) that minimises the estimated DRAM bytes of the
+// operands.  The c tiles in flight span mw m blocks and nw n blocks: n
+// fastest (gm = 1) gives mw = ceil(c / Nt), nw = min(Nt, c); strips of gm
+// give mw = min(gm, c), nw = min(Nt, ceil(c / gm)).  A (a_bytes in total) is
+// then read about Nt / nw times and B about Mt / mw times, except that an
+// operand small enough to stay in L2 (48 MB) is read once.  Candidates: 1
+// and all m blocks.
+int pick_strip(int Mt, int Nt, int c, double a_bytes, double b_bytes) {
+  constexpr double kL2Resident = 48.0 * 1024 * 1024;
+  auto cost = [&](int gm) {
+    double mw, nw;
+    if (gm == 1) {
+      mw = (c + Nt - 1) / Nt;
+      nw = Nt < c ? Nt : c;
+    } else {
+      mw = gm < c ? gm : c;
+      const int n = (c + gm - 1) / gm;
+      nw = n < Nt ? n : Nt;
+    }
+    const double a_reads = (a_bytes <= kL2Resident) ? 1.0 : (Nt / nw > 1.0 ? Nt / nw : 1.0);
+    const double b_reads = (b_bytes <= kL2Resident) ? 1.0 : (Mt / mw > 1.0 ? Mt / mw : 1.0);
+    return a_bytes * a_reads + b_bytes * b_reads;
+  };
+  return cost(Mt) < cost(1) ? Mt : 1;
+}
+
 template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI>
 cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int splits, int num_sms,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, double a_bytes, double b_bytes) {
   using C = Cfg2<kI8, kAMN, kBMN, STAGES>;
   auto kern = tc_gemm_pair_kernel<kI8, kAMN, kBMN, STAGES, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -600,6 +634,7 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArg
   sc.total = sc.Mt * sc.Nt * splits;
   int pairs = num_sms / 2;
   if (pairs > sc.total) pairs = sc.total;
+  sc.GM = pick_strip(sc.Mt, sc.Nt, pairs, a_bytes, b_bytes);
   kern<<<2 * pairs, kThreads, C::SMEM_BYTES, stream>>>(ta, tb, a, sc);
   return cudaGetLastError();
 }
@@ -644,7 +679,10 @@ cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_
   a.amax = amax;
   a.gamma = gamma;
   a.err = err;
-  if (use_pair) return run_pair<true, false, false, kPairStages, kEpiFwd>(ta, tb, a, 1, num_sms, stream);
+  if (use_pair)
+    return run_pair<true, false, false, kPairStages, kEpiFwd>(ta, tb, a, 1, num_sms, stream,
+                                                             static_cast<double>(T) * d_in,
+                                                             static_cast<double>(d_out) * d_in);
   return run<true, false, false, kBN, kStages, kEpiFwd>(ta, tb, a, 1, num_sms, stream);
 }
 
@@ -670,7 +708,8 @@ cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf1
       a.ldo = d_in;
       a.gamma = gamma;
       a.err = err;
-      e = use_pair ? run_pair<false, false, true, kPairStages, kEpiDx>(ta, tb, a, 1, num_sms, stream)
+      e = use_pair ? run_pair<false, false, true, kPairStages, kEpiDx>(ta, tb, a, 1, num_sms, stream,
+                                                                      2.0 * T * d_out, 2.0 * d_out * d_in)
                    : run<false, false, true, kBN, kStages, kEpiDx>(ta, tb, a, 1, num_sms, stream);
     }
     if (e != cudaSuccess) return e;
@@ -706,7 +745,8 @@ cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf1
       e = cudaMemsetAsync(dW, 0, sizeof(float) * static_cast<size_t>(d_out) * d_in, stream);
       if (e != cudaSuccess) return e;
     }
-    e = use_pair ? run_pair<false, true, true, kPairStages, kEpiDw>(ta, tb, a, splits, num_sms, stream)
+    e = use_pair ? run_pair<false, true, true, kPairStages, kEpiDw>(ta, tb, a, splits, num_sms, stream,
+                                                                   2.0 * T * d_out, 2.0 * T * d_in)
                  : run<false, true, true, kBN, kStages, kEpiDw>(ta, tb, a, splits, num_sms, stream);
   }
   return e;
