@@ -364,6 +364,28 @@ def run_decode(args):
                       "peak_source": pkk["src"], "results": results}))
 
 
+# ----------------------------------------------------------------- ranks
+def rank_env():
+    """(rank, world_size, local_rank) from the torchrun environment (1 process: 0, 1, 0)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value, dist=None, device="cpu"):
+    """The largest `value` over all ranks (the job's time is its slowest rank's)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(world, tokens_per_rank, ms_per_step):
+    """Whole-job tokens/s: every rank runs its own batch (weak scaling) and the
+    step time is the maximum over ranks."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ----------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -382,9 +404,7 @@ def main():
         run_decode(args)
         return
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local_rank = rank_env()
     ls = synth.layer_set(args.workload)
     T = args.tokens or WORKLOADS[args.workload][0]
     dist_name, outl, ties = WORKLOADS[args.workload][1:]
@@ -452,13 +472,9 @@ def main():
         stream.synchronize()
     barrier()
     sbl.sbl_check(stream)
-    elapsed_ms = start.elapsed_time(end)
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = t.item()
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dist, "cuda")
     ms_per_step = elapsed_ms / args.steps
-    value = world * T / (ms_per_step / 1e3)
+    value = job_throughput(world, T, ms_per_step)
 
     per_call = {k: sum(a.elapsed_time(b) for a, b in v) / args.steps for k, v in ev.items()}
     launches = {k: len(v) // args.steps for k, v in ev.items()}
@@ -482,12 +498,8 @@ def main():
                 h.copy_(d, non_blocking=True)
     e1.record(stream)
     stream.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / max(1, args.e2e_steps)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
-    e2e_value = world * T / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(1, args.e2e_steps), dist, "cuda")
+    e2e_value = job_throughput(world, T, e2e_ms)
 
     # ---- roofline of the dominant call family and of the whole step
     pk = peaks()
