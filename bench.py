@@ -364,6 +364,83 @@ def run_decode(args):
                       "peak_source": pkk["src"], "results": results}))
 
 
+# ----------------------------------------------------------------- prefill
+def run_prefill(args):
+    """Prefill forward on the packed 6:8 format of the 3B layer set: per
+    projection, int8 activations (absmax-quantised N(0, 1)) times the packed
+    weight expanded in shared memory (sbl_forward_packed), against the same
+    product from the unpacked int8 W_eff (sbl_forward).  Shapes: 512 tokens
+    (1 x 512), 8192 (8 x 1024) and 32768 (16 x 2048).  One pass = the seven
+    projections; int8 ops = 2 T P (dense-equivalent)."""
+    import semi_structured_sparsity_step_b200 as sbl
+    from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer, act_quant
+    torch.cuda.set_device(0)
+    ls = synth.layer_set("qwen2.5-3b")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    layers = []
+    for i, p in enumerate(ls.projections):
+        w = make_weight(ls, i, p).cuda()
+        L = SparseBitLinearLayer(w, N_KEEP, M_GROUP)
+        L.weight_step()
+        nbytes = sbl.sbl_packed_bytes(p.d_out, p.d_in, N_KEEP, M_GROUP)
+        pk = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        sbl.sbl_pack(L.W_eff, p.d_out, p.d_in, N_KEEP, M_GROUP, pk, nbytes)
+        layers.append((p, L, pk))
+    sbl.sbl_check()
+    pk_peak = peaks()
+    i8_peak = pk_peak["bf16"] * NOMINAL_I8_OVER_BF16  # burst: each pass is timed on its own
+    results = {}
+    stream = torch.cuda.Stream()
+    for T in (512, 8192, 32768):
+        xs = {}
+        for n, d in ls.inputs.items():
+            x = torch.randn(T, d, generator=g, device="cuda").to(torch.bfloat16)
+            xq = torch.empty(T, d, dtype=torch.int8, device="cuda")
+            am = torch.empty(T, dtype=torch.float32, device="cuda")
+            act_quant(x, xq, am)
+            xs[n] = (xq, am)
+        ys = [torch.empty(T, p.d_out, dtype=torch.float32, device="cuda") for (p, _, _) in layers]
+
+        def one_pass(packed):
+            for (p, L, pk), y in zip(layers, ys):
+                xq, am = xs[p.input_name]
+                if packed:
+                    sbl.sbl_forward_packed(xq, am, pk, L.gamma, T, p.d_in, p.d_out, N_KEEP, M_GROUP, y, None, stream)
+                else:
+                    sbl.sbl_forward(xq, am, L.W_eff, L.gamma, T, p.d_in, p.d_out, y, None, stream)
+
+        row = {}
+        for packed in (True, False):
+            with torch.cuda.stream(stream):
+                for _ in range(args.warmup):
+                    one_pass(packed)
+            stream.synchronize()
+            reps = max(args.steps, 5)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            with torch.cuda.stream(stream):
+                for _ in range(reps):
+                    one_pass(packed)
+            e1.record(stream)
+            stream.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            tops = 2.0 * T * ls.params / (ms / 1e3) / 1e12
+            row["packed" if packed else "int8_weff"] = {"ms_per_pass": ms, "tokens_per_s": T / (ms / 1e3),
+                                                         "int8_tops": tops, "frac_int8_peak": tops / i8_peak}
+        sbl.sbl_check()
+        results[str(T)] = row
+        del xs, ys
+        torch.cuda.empty_cache()
+    print(json.dumps({"metric": "Sparse-BitLinear prefill forward on the packed 6:8 format (3B layer set)",
+                      "unit": "tokens/s", "peak_int8_tops": i8_peak,
+                      "peak_source": f"{pk_peak['src']} bf16 burst x2 nominal int8/bf16",
+                      "workload": "qwen2.5-3b layer set, 6:8 packed (2.5 bit/weight), T = 512 / 8192 / 32768, "
+                                  "Xq from absmax-quantised N(0,1), fp32 outputs",
+                      "results": results}))
+
+
 # ----------------------------------------------------------------- ranks
 def rank_env():
     """(rank, world_size, local_rank) from the torchrun environment (1 process: 0, 1, 0)."""
@@ -397,11 +474,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen2.5-3b")
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (0: the workload's default)")
-    ap.add_argument("--mode", choices=["train", "decode"], default="train")
+    ap.add_argument("--mode", choices=["train", "decode", "prefill"], default="train")
     ap.add_argument("--layers", type=int, default=36, help="decode mode: distinct layer sets in the stack")
     args = ap.parse_args()
     if args.mode == "decode":
         run_decode(args)
+        return
+    if args.mode == "prefill":
+        run_prefill(args)
         return
 
     rank, world, local_rank = rank_env()

@@ -158,6 +158,18 @@ sbl_status sbl_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff,
                        const float* gamma, int T, int d_in, int d_out, float* Y,
                        int32_t* acc, void* stream);
 
+/* Forward product with the weight read from the packed format (prefill on a
+ * deployed model): the same result as sbl_forward on the unpacked W_eff, bit
+ * for bit.  [summary] Algorithm 1 step (6); [article] 7.1 (cached sparse
+ * format); the packed weight is expanded tile by tile into shared memory
+ * right before the int8 tensor-core MMA, so HBM only carries 2.5 bit/weight
+ * at 6:8.
+ *   packed  sbl_pack output of the [d_out, d_in] weight, N:M as packed.
+ *   other arguments as sbl_forward. */
+sbl_status sbl_forward_packed(const int8_t* Xq, const float* amax, const uint8_t* packed,
+                              const float* gamma, int T, int d_in, int d_out, int N, int M,
+                              float* Y, int32_t* acc, void* stream);
+
 /* ------------------------------------------------------------------------
  * Dual-STE backward on bf16 tensor cores (tcgen05, fp32 accumulation).
  * [summary] 前置知识 / STE and 核心方法 (masked weights receive the full

@@ -36,6 +36,7 @@ SIGNATURES = {
     "sbl_mask_quant_noalloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp]),
     "sbl_act_quant": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_forward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
+    "sbl_forward_packed": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_backward_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
     "sbl_backward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp, _c_size, _vp]),
     "sbl_packed_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
@@ -145,6 +146,11 @@ def sbl_act_quant(X, T, d_in, Xq, amax, stream=None) -> None:
 def sbl_forward(Xq, amax, W_eff, gamma, T, d_in, d_out, Y, acc=None, stream=None) -> None:
     _call("sbl_forward", _ptr(Xq), _ptr(amax), _ptr(W_eff), _ptr(gamma), T, d_in, d_out, _ptr(Y), _ptr(acc),
           _stream(stream))
+
+
+def sbl_forward_packed(Xq, amax, packed, gamma, T, d_in, d_out, N, M, Y, acc=None, stream=None) -> None:
+    _call("sbl_forward_packed", _ptr(Xq), _ptr(amax), _ptr(packed), _ptr(gamma), T, d_in, d_out, N, M, _ptr(Y),
+          _ptr(acc), _stream(stream))
 
 
 def sbl_backward_workspace_bytes(T, d_in, d_out) -> int:

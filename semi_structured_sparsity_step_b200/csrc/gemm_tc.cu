@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   empty[s]  (both CTAs): freed by one multicast tcgen05.commit.
 //   tfull[b]  (both CTAs): accumulator buffer b ready (multicast commit).
 //   tempty[b] (even CTA only): 4 epilogue warps of each CTA arrive.
-template <bool kI8, bool kAMN, bool kBMN, int STAGES>
+template <bool kI8, bool kAMN, bool kBMN, int STAGES, int KP = 0>
 struct Cfg2 {
   static constexpr int BN = 256;                 // N of the pair's tile
   static constexpr int BK = kI8 ? 128 : 64;      // elements per stage along K (128 bytes)
@@ -337,16 +337,101 @@ struct Cfg2 {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int EPI_WARP_FLOATS = 32 * 33;
   static constexpr int EPI_BYTES = 4 * EPI_WARP_FLOATS * 4;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256;
+  // Packed B (KP > 0): per-lane replicated decode tables after the barriers.
+  static constexpr int LUT_BYTES = KP > 0 ? (64 + 256) * 32 * 4 : 0;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256 + LUT_BYTES;
+  static constexpr int THREADS = KP > 0 ? 448 : 192;  // packed: + 8 decoder warps
   static constexpr uint32_t TMEM_COLS = 2 * BN;
   static constexpr uint32_t IDESC = instr_desc(kI8, 256, BN, kAMN, kBMN);
 };
 
-template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// Where the packed weight lives (forward from the packed format).
+struct PackedB {
+  const uint8_t* codes;  // codes plane, row stride crow
+  const uint8_t* index;  // index plane, row stride irow
+  long long crow, irow;
+  int rows;              // d_out
+};
+
+__device__ __forceinline__ uint32_t packed_code_byte(uint32_t code) {
+  return code == 1u ? 0x01u : (code == 3u ? 0xFFu : 0u);
+}
+
+// Decodes half `hf` (chunks 8 hf .. 8 hf + 7, 64 weights) of K block `kb`
+// of weight row `row` from the packed planes into row `r` of a 128 x
+// 128-byte int8 B tile with the 128-byte swizzle (16-byte unit c of row r
+// stored at unit c ^ (r % 8)), the layout a TMA load of W_eff would produce.
+// Chunks past d_in/8 and rows past d_out decode to zeros.  Tables are
+// replicated per lane (entry e of copy l at word e * 32 + l).
+template <int KP>
+struct PackedHalf {
+  uint32_t w[(KP + 1) / 2 + 1];  // 8 chunks x 2KP bits = 2KP bytes (+1 word of zeros)
+  uint2 m;                       // the 8 slot masks
+};
+
+template <int KP>
+__device__ __forceinline__ void load_packed_half(PackedHalf<KP>& ph, const PackedB& pb, int row, int kb, int hf,
+                                                 int nchunks) {
+  uint32_t* w = ph.w;
+#pragma unroll
+  for (int i = 0; i < (KP + 1) / 2 + 1; ++i) w[i] = 0u;
+  uint2 m = make_uint2(0u, 0u);
+  const int ch0 = kb * 16 + 8 * hf;
+  if (row < pb.rows && ch0 < nchunks) {
+    const int valid = (nchunks * 2 * KP + 7) / 8;  // code bytes of a row
+    const uint8_t* cr = pb.codes + static_cast<long long>(row) * pb.crow;
+    const int off = ch0 * 2 * KP / 8;              // 2KP bytes per 8 chunks
+    if constexpr ((KP & 1) == 0) {
+#pragma unroll
+      for (int i = 0; i < KP / 2; ++i)
+        if (off + 4 * i < valid) w[i] = __ldg(reinterpret_cast<const uint32_t*>(cr + off) + i);
+    } else {
+#pragma unroll
+      for (int i = 0; i < KP; ++i)
+        if (off + 2 * i < valid)
+          w[i >> 1] |= static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(cr + off) + i)) << (16 * (i & 1));
+    }
+    m = __ldg(reinterpret_cast<const uint2*>(pb.index + static_cast<long long>(row) * pb.irow + ch0));
+  }
+  ph.m = m;
+}
+
+template <int KP>
+__device__ __forceinline__ void expand_packed_half(const PackedHalf<KP>& ph, int hf, uint8_t* tile, int r,
+                                                   const uint32_t* s_code, const uint32_t* s_sel, int lane) {
+  const uint32_t* w = ph.w;
+  const uint2 m = ph.m;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t out[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = 2 * c + h;  // chunk within the half
+      const int bit = 2 * KP * j;
+      const uint32_t v = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31);
+      const uint32_t codes = (2 * KP == 32) ? v : (v & ((1u << (2 * KP)) - 1u));
+      const uint32_t mask = ((j < 4 ? m.x : m.y) >> (8 * (j & 3))) & 0xFFu;
+      uint32_t lo = s_code[((codes & 63u) << 5) + lane], hi = 0u;
+      if constexpr (KP > 3) {
+        const uint32_t t1 = s_code[(((codes >> 6) & 63u) << 5) + lane];
+        lo |= t1 << 24;
+        hi = t1 >> 8;
+        if constexpr (KP > 6) hi |= s_code[(((codes >> 12) & 63u) << 5) + lane] << 16;
+      }
+      const uint32_t sel = s_sel[(mask << 5) + lane];
+      out[2 * h] = __byte_perm(lo, hi, sel & 0xFFFFu);
+      out[2 * h + 1] = __byte_perm(lo, hi, sel >> 16);
+    }
+    const int unit = 4 * hf + c;  // 16-byte unit within the 128-byte row
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((unit ^ (r & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI, int KP = 0>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmArgs args, const Sched sched) {
-  using C = Cfg2<kI8, kAMN, kBMN, STAGES>;
+                        const GemmArgs args, const Sched sched, const PackedB pb) {
+  using C = Cfg2<kI8, kAMN, kBMN, STAGES, KP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* epi_tiles = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES);
@@ -356,6 +441,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* s_code = reinterpret_cast<uint32_t*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES + 256);  // KP > 0
+  uint32_t* s_sel = s_code + 64 * 32;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -366,9 +453,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int KB = (args.K + C::BK - 1) / C::BK;
   const uint32_t peer_abort = pair::map_to(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
 
+  if constexpr (KP > 0) {
+    for (int i = threadIdx.x; i < 64 * 32; i += blockDim.x) {
+      const uint32_t c = static_cast<uint32_t>(i) >> 5;
+      s_code[i] = packed_code_byte(c & 3u) | (packed_code_byte((c >> 2) & 3u) << 8) |
+                  (packed_code_byte((c >> 4) & 3u) << 16);
+    }
+    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
+      const uint32_t c = static_cast<uint32_t>(i) >> 5;
+      uint32_t sel = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t nib = ((c >> q) & 1u) ? static_cast<uint32_t>(__popc(c & ((1u << q) - 1u))) : 7u;
+        sel |= nib << (4 * q);
+      }
+      s_sel[i] = sel;
+    }
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      // packed B: the even CTA's producer plus 8 decoder warps of each CTA
+      mbar_init(&full[s], KP > 0 ? 17 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -378,14 +483,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    if constexpr (KP == 0) tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
     pair::tmem_alloc(tmem_slot, C::TMEM_COLS);
     pair::tmem_relinquish();
   }
   tc_fence_before();
-  pair::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+  pair::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated, tables built
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -413,7 +518,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(&full[s], KP > 0 ? 2 * C::A_BYTES : 2 * C::STAGE_BYTES);
           const uint32_t fbar = pair::map_to(smem_u32(&full[s]), 0u);
           uint8_t* sa = smem + s * C::STAGE_BYTES;
           uint8_t* sb = sa + C::A_BYTES;
@@ -424,11 +529,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             pair::tma_load_2d(sa, &tmA, fbar, m0, kc);
             pair::tma_load_2d(sa + C::BK * 128, &tmA, fbar, m0 + 64, kc);
           }
-          if constexpr (!kBMN) {
-            pair::tma_load_2d(sb, &tmB, fbar, kc, n0);
-          } else {
-            pair::tma_load_2d(sb, &tmB, fbar, n0, kc);
-            pair::tma_load_2d(sb + C::BK * 128, &tmB, fbar, n0 + 64, kc);
+          if constexpr (KP == 0) {
+            if constexpr (!kBMN) {
+              pair::tma_load_2d(sb, &tmB, fbar, kc, n0);
+            } else {
+              pair::tma_load_2d(sb, &tmB, fbar, n0, kc);
+              pair::tma_load_2d(sb + C::BK * 128, &tmB, fbar, n0 + 64, kc);
+            }
           }
           ++it;
         }
@@ -477,6 +584,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ++it;
         }
         pair::umma_commit_multicast(&tfull[b], 0x3);
+      }
+    }
+  } else if (KP > 0 && warp >= 6) {
+    if constexpr (KP > 0) {
+      // Decoder warps 6-13: thread (r, hf) expands half hf of row r of this
+      // CTA's 128-row B half for every K block, one stage ahead of the MMA
+      // like the TMA producer.
+      const int dt = (warp - 6) * 32 + lane;
+      const int r = dt & 127, hf = dt >> 7;
+      const int nchunks = args.K / 8;
+      // Walk the same (item, k block) sequence as the TMA producer; the
+      // packed words of the next k block are loaded (from L2) into registers
+      // before waiting for the current stage, hiding the load latency.
+      int w = pair_id, kb = 0, kb1 = 0, row = 0;
+      auto start_item = [&](int item) {
+        int mb, nb, sp;
+        sched.item(item, mb, nb, sp);
+        kb = sp * args.kb_per_split;
+        kb1 = min(KB, kb + args.kb_per_split);
+        row = nb * C::BN + 128 * static_cast<int>(rank) + r;
+      };
+      if (w < sched.total) start_item(w);
+      PackedHalf<KP> cur, nxt;
+      if (w < sched.total) load_packed_half<KP>(cur, pb, row, kb, hf, nchunks);
+      int it = 0;
+      while (w < sched.total) {
+        // position of the next k block in the sequence
+        int nw = w, nkb = kb + 1, nkb1 = kb1, nrow = row;
+        if (nkb >= kb1) {
+          nw = w + n_pairs;
+          if (nw < sched.total) {
+            int mb, nb, sp;
+            sched.item(nw, mb, nb, sp);
+            nkb = sp * args.kb_per_split;
+            nkb1 = min(KB, nkb + args.kb_per_split);
+            nrow = nb * C::BN + 128 * static_cast<int>(rank) + r;
+          }
+        }
+        if (nw < sched.total) load_packed_half<KP>(nxt, pb, nrow, nkb, hf, nchunks);
+        const int s = it % STAGES;
+        const uint32_t round = static_cast<uint32_t>(it / STAGES);
+        const bool waited = mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, args.err);
+        if (!__all_sync(0xFFFFFFFFu, waited)) {  // the whole warp leaves together
+          give_up();
+          break;
+        }
+        uint8_t* sb = smem + s * C::STAGE_BYTES + C::A_BYTES;
+        expand_packed_half<KP>(cur, hf, sb, r, s_code, s_sel, lane);
+        // make the generic-proxy stores visible to the tensor core (async proxy)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t fb = pair::map_to(smem_u32(&full[s]), 0u);
+          asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(fb) : "memory");
+        }
+        ++it;
+        w = nw;
+        kb = nkb;
+        kb1 = nkb1;
+        row = nrow;
+        cur = nxt;
       }
     }
   } else {
@@ -620,11 +788,11 @@ int pick_strip(int Mt, int Nt, int c, double a_bytes, double b_bytes) {
   return cost(Mt) < cost(1) ? Mt : 1;
 }
 
-template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI>
+template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI, int KP = 0>
 cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int splits, int num_sms,
-                     cudaStream_t stream, double a_bytes, double b_bytes) {
-  using C = Cfg2<kI8, kAMN, kBMN, STAGES>;
-  auto kern = tc_gemm_pair_kernel<kI8, kAMN, kBMN, STAGES, EPI>;
+                     cudaStream_t stream, double a_bytes, double b_bytes, const PackedB& pb = PackedB{}) {
+  using C = Cfg2<kI8, kAMN, kBMN, STAGES, KP>;
+  auto kern = tc_gemm_pair_kernel<kI8, kAMN, kBMN, STAGES, EPI, KP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   Sched sc;
@@ -635,13 +803,14 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArg
   int pairs = num_sms / 2;
   if (pairs > sc.total) pairs = sc.total;
   sc.GM = pick_strip(sc.Mt, sc.Nt, pairs, a_bytes, b_bytes);
-  kern<<<2 * pairs, kThreads, C::SMEM_BYTES, stream>>>(ta, tb, a, sc);
+  kern<<<2 * pairs, C::THREADS, C::SMEM_BYTES, stream>>>(ta, tb, a, sc, pb);
   return cudaGetLastError();
 }
 
 constexpr int kBN = 256;
 constexpr int kStages = 4;
 constexpr int kPairStages = 6;
+constexpr int kPackedStages = 4;
 
 }  // namespace
 
@@ -750,6 +919,55 @@ cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf1
                  : run<false, true, true, kBN, kStages, kEpiDw>(ta, tb, a, splits, num_sms, stream);
   }
   return e;
+}
+
+cudaError_t launch_forward_packed(const int8_t* Xq, const float* amax, const uint8_t* packed, const float* gamma,
+                                  int T, int d_in, int d_out, int N, int M, float* Y, int32_t* acc,
+                                  cudaStream_t stream, int num_sms, uint32_t* err) {
+  if (T == 0 || d_out == 0) return cudaSuccess;
+  if (d_in == 0) {
+    cudaError_t e = cudaMemsetAsync(Y, 0, sizeof(float) * static_cast<size_t>(T) * d_out, stream);
+    if (e == cudaSuccess && acc != nullptr)
+      e = cudaMemsetAsync(acc, 0, sizeof(int32_t) * static_cast<size_t>(T) * d_out, stream);
+    return e;
+  }
+  CUtensorMap ta;
+  if (!make_tmap(&ta, Xq, false, d_in, T, d_in, 128, BM)) return cudaErrorInvalidValue;
+  GemmArgs a{};
+  a.M = T;
+  a.N = d_out;
+  a.K = d_in;
+  a.kb_per_split = (d_in + 127) / 128;
+  a.out = Y;
+  a.ldo = d_out;
+  a.acc_out = acc;
+  a.amax = amax;
+  a.gamma = gamma;
+  a.err = err;
+  PackedB pb{};
+  pb.crow = static_cast<long long>(packed_codes_row_bytes(d_in, N, M));
+  pb.irow = static_cast<long long>(packed_index_row_bytes(d_in, M));
+  pb.codes = packed;
+  pb.index = packed + static_cast<size_t>(d_out) * pb.crow;
+  pb.rows = d_out;
+  const double ab = static_cast<double>(T) * d_in;
+  const double bb = static_cast<double>(d_out) * (pb.crow + pb.irow);
+  switch (8 * N / M) {
+#define SBL_FWD_PACKED(KK) \
+  case KK:                 \
+    return run_pair<true, false, false, kPackedStages, kEpiFwd, KK>(ta, ta, a, 1, num_sms, stream, ab, bb, pb);
+    SBL_FWD_PACKED(1)
+    SBL_FWD_PACKED(2)
+    SBL_FWD_PACKED(3)
+    SBL_FWD_PACKED(4)
+    SBL_FWD_PACKED(5)
+    SBL_FWD_PACKED(6)
+    SBL_FWD_PACKED(7)
+    SBL_FWD_PACKED(8)
+#undef SBL_FWD_PACKED
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace sbl

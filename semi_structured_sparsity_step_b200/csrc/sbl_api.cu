@@ -170,6 +170,24 @@ sbl_status sbl_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff,
                                   d->num_sms, d->err));
 }
 
+sbl_status sbl_forward_packed(const int8_t* Xq, const float* amax, const uint8_t* packed, const float* gamma,
+                              int T, int d_in, int d_out, int N, int M, float* Y, int32_t* acc, void* stream) {
+  sbl_status st = check_nm(N, M);
+  if (st != SBL_OK) return st;
+  if ((st = check_dims(d_in, d_out)) != SBL_OK) return st;
+  if (T < 0 || d_in % M != 0) return SBL_ERR_SHAPE;
+  if (T == 0 || d_out == 0) return SBL_OK;
+  if (Xq == nullptr || amax == nullptr || packed == nullptr || gamma == nullptr || Y == nullptr)
+    return SBL_ERR_INVALID_ARG;
+  if (!aligned16(Xq) || !aligned16(amax) || !aligned16(packed) || !aligned16(Y) || !aligned16(acc) ||
+      (reinterpret_cast<uintptr_t>(gamma) & 3u) != 0)
+    return SBL_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  return from_cuda(launch_forward_packed(Xq, amax, packed, gamma, T, d_in, d_out, N, M, Y, acc,
+                                         static_cast<cudaStream_t>(stream), d->num_sms, d->err));
+}
+
 size_t sbl_backward_workspace_bytes(int T, int d_in, int d_out) {
   (void)T;
   (void)d_in;

@@ -38,6 +38,9 @@ extern int g_gemm_variant;
 cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
                            int d_in, int d_out, float* Y, int32_t* acc, cudaStream_t stream, int num_sms,
                            uint32_t* err);
+cudaError_t launch_forward_packed(const int8_t* Xq, const float* amax, const uint8_t* packed, const float* gamma,
+                                  int T, int d_in, int d_out, int N, int M, float* Y, int32_t* acc,
+                                  cudaStream_t stream, int num_sms, uint32_t* err);
 cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf16, const float* gamma, int T,
                             int d_in, int d_out, float* dX, float* dW, int accumulate_dW, cudaStream_t stream,
                             int num_sms, uint32_t* err);

@@ -273,3 +273,28 @@ def test_gemv_group_matches_single_calls(lib):
     lib.sbl_check()
     for (_, _, _, _, Y, _, _), ref in zip(probs, refs):
         assert np.array_equal(Y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("T,d_out,d_in,N,M", [
+    (64, 256, 256, 6, 8), (300, 264, 2064, 6, 8), (129, 520, 1040, 2, 4), (257, 136, 400, 4, 8),
+    (100, 392, 2048, 8, 8), (33, 8, 4864, 1, 8), (77, 128, 272, 3, 4),
+])
+def test_forward_from_packed_matches_oracle(lib, T, d_out, d_in, N, M):
+    """The forward that expands the packed weight in shared memory gives the
+    oracle's int32 accumulators and outputs (and so sbl_forward's)."""
+    w = synth.trimodal_weight(d_out, d_in, seed=40, tensor_id=T)
+    x = synth.activations(T, d_in, seed=40, tensor_id=100 + T, outlier_frac=0.01)
+    weff, gamma, _ = oracle.effective_weight(synth.bits(w), N, M)
+    xq, amax = oracle.act_quant(synth.bits(x))
+    nbytes = lib.sbl_packed_bytes(d_out, d_in, N, M)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    lib.sbl_pack(torch.from_numpy(weff).cuda(), d_out, d_in, N, M, packed, nbytes)
+    Y = torch.empty(T, d_out, dtype=torch.float32, device="cuda")
+    acc = torch.empty(T, d_out, dtype=torch.int32, device="cuda")
+    g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+    lib.sbl_forward_packed(torch.from_numpy(xq).cuda(), torch.from_numpy(amax).cuda(), packed, g, T, d_in, d_out, N,
+                           M, Y, acc)
+    lib.sbl_check()
+    racc = oracle.forward_acc(xq, weff)
+    assert np.array_equal(acc.cpu().numpy(), racc)
+    assert np.array_equal(Y.cpu().numpy(), oracle.forward_out(racc, gamma, amax))
