@@ -305,3 +305,124 @@ def gemv_packed(xq: np.ndarray, amax: np.ndarray, packed: np.ndarray,
     """y = forward_out(X_q . unpack(packed)^T, gamma, amax)."""
     w = unpack(packed, d_out, d_in, N, M)
     return forward_out(forward_acc(xq, w), gamma, amax)
+
+
+# --------------------------------------------------------------------------
+# (a8) 2:4 compressed weight for the sparse tensor core
+# [summary] 前置知识 / 半结构化 N:M 稀疏 (2:4 -- two kept of every four --
+# is the pattern NVIDIA's sparse tensor cores accelerate) and 核心方法
+# (masking after quantisation keeps the deployed weight N:M-structured so it
+# can go to the sparse tensor core as it is).
+#
+# The format (this library's, the pages fix none) has two planes:
+#   values plane: d_out rows of vrow = ceil16(d_in / 2) bytes; row o holds,
+#     for every group g of four weights, the int8 values of its two slots in
+#     ascending position order at bytes 2g and 2g + 1; bytes past d_in / 2
+#     are zero;
+#   selector plane (from the first 1024-byte boundary at or after the end
+#     of the values plane): for every row and group a 4-bit selector
+#     i0 | (i1 << 2), i0 < i1 the two slot positions.  It is tiled for the
+#     tensor core: blocks of 128 rows x 256 weights (4096 bytes), block
+#     (mb, kb) at (mb * KB + kb) * 4096; inside a block, two halves of 128
+#     weights each (2048 bytes), row r of a half at 16 r, and the selector of
+#     group j of that half in byte j // 2, low nibble for even j.  Rows are
+#     padded to a multiple of 256 and weights to a multiple of 256; padding
+#     groups get the selector of slots (0, 1) and zero values.
+# Slots are the group's nonzero positions plus, if fewer than two, its
+# lowest zero positions (the rule of the packed format above).
+# --------------------------------------------------------------------------
+SP24_PAD_NIBBLE = 0x4   # slots (0, 1)
+
+
+def sparse24_layout(d_out: int, d_in: int):
+    """(vrow, meta_off, total_bytes, KB, MB): values row bytes, selector-plane
+    offset, buffer size, 256-weight blocks per row, 128-row blocks."""
+    vrow = _ceil16(d_in // 2)
+    KB = -(-d_in // 256)
+    MB = 2 * (-(-d_out // 256))
+    meta_off = -(-(d_out * vrow) // 1024) * 1024
+    return vrow, meta_off, meta_off + MB * KB * 4096, KB, MB
+
+
+def _selector_plane(nib: np.ndarray, KB: int, MB: int) -> np.ndarray:
+    """Selector nibbles on the padded grid [MB * 128, KB * 64] -> the plane's
+    bytes: two groups per byte (low nibble = even group), then the blocks of
+    128 rows x 256 weights in (mb, kb) order, each as two halves of 128 rows
+    x 16 bytes."""
+    byte = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)          # [MB*128, KB*32]
+    blocks = byte.reshape(MB, 128, KB, 2, 16).transpose(0, 2, 3, 1, 4)    # mb, kb, half, r, q
+    return np.ascontiguousarray(blocks).reshape(-1)
+
+
+def _selector_grid(plane: np.ndarray, KB: int, MB: int) -> np.ndarray:
+    """Inverse of :func:`_selector_plane`: nibbles [MB * 128, KB * 64]."""
+    byte = plane.reshape(MB, KB, 2, 128, 16).transpose(0, 3, 1, 2, 4).reshape(MB * 128, KB * 32)
+    nib = np.empty((MB * 128, KB * 64), dtype=np.uint8)
+    nib[:, 0::2] = byte & 0xF
+    nib[:, 1::2] = byte >> 4
+    return nib
+
+
+def compress24(weff: np.ndarray) -> np.ndarray:
+    """W_eff (int8 [d_out, d_in], at most two nonzeros per group of four)
+    -> the compressed buffer (uint8)."""
+    d_out, d_in = weff.shape
+    assert d_in % 4 == 0
+    vrow, meta_off, total, KB, MB = sparse24_layout(d_out, d_in)
+    G = d_in // 4
+    grp = weff.reshape(d_out, G, 4).astype(np.int64)
+    nz = grp != 0
+    if (nz.sum(axis=-1) > 2).any():
+        o, g = np.argwhere(nz.sum(axis=-1) > 2)[0]
+        raise ValueError(f"row {o} group {g}: more than 2 nonzeros")
+    # nonzero positions first, then zero positions, each by index; take two
+    key = np.where(nz, 0, 4) + np.arange(4)
+    slots = np.sort(np.argsort(key, axis=-1)[..., :2], axis=-1)      # [d_out, G, 2]
+    vals = np.take_along_axis(grp, slots, axis=-1).astype(np.int8)    # [d_out, G, 2]
+    out = np.zeros(total, dtype=np.uint8)
+    vplane = np.zeros((d_out, vrow), dtype=np.uint8)
+    vplane[:, :2 * G] = vals.reshape(d_out, 2 * G).view(np.uint8)
+    out[:d_out * vrow] = vplane.reshape(-1)
+    nib = np.full((MB * 128, KB * 64), SP24_PAD_NIBBLE, dtype=np.uint8)
+    nib[:d_out, :G] = slots[..., 0] | (slots[..., 1] << 2)
+    out[meta_off:] = _selector_plane(nib, KB, MB)
+    return out
+
+
+def _selectors(buf: np.ndarray, d_out: int, d_in: int):
+    """(i0, i1) arrays [d_out, d_in / 4] read back from the selector plane."""
+    vrow, meta_off, total, KB, MB = sparse24_layout(d_out, d_in)
+    nib = _selector_grid(buf[meta_off:], KB, MB)[:d_out, :d_in // 4]
+    return nib & 3, nib >> 2
+
+
+def decompress24(buf: np.ndarray, d_out: int, d_in: int) -> np.ndarray:
+    """Inverse of :func:`compress24` (raises on a selector with i0 >= i1)."""
+    vrow, meta_off, total, KB, MB = sparse24_layout(d_out, d_in)
+    assert buf.size == total
+    G = d_in // 4
+    i0, i1 = _selectors(buf, d_out, d_in)
+    if (i0 >= i1).any():
+        raise ValueError("selector with i0 >= i1")
+    vals = buf[:d_out * vrow].reshape(d_out, vrow)[:, :2 * G].view(np.int8).reshape(d_out, G, 2)
+    w = np.zeros((d_out, G, 4), dtype=np.int8)
+    o_idx, g_idx = np.meshgrid(np.arange(d_out), np.arange(G), indexing="ij")
+    w[o_idx, g_idx, i0] = vals[..., 0]
+    w[o_idx, g_idx, i1] = vals[..., 1]
+    return w.reshape(d_out, d_in)
+
+
+def forward_acc_sparse24(xq: np.ndarray, buf: np.ndarray, d_out: int, d_in: int) -> np.ndarray:
+    """acc[t, o] = sum_g sum_s value[o, g, s] * xq[t, 4 g + i_s[o, g]]: the
+    product as a sparse tensor core forms it, from the two kept values of
+    each group and the activations its selector picks (exact integers)."""
+    vrow, meta_off, total, KB, MB = sparse24_layout(d_out, d_in)
+    G = d_in // 4
+    i0, i1 = _selectors(buf, d_out, d_in)
+    vals = buf[:d_out * vrow].reshape(d_out, vrow)[:, :2 * G].view(np.int8).reshape(d_out, G, 2).astype(np.int64)
+    xg = xq.astype(np.int64).reshape(xq.shape[0], G, 4)
+    acc = np.zeros((xq.shape[0], d_out), dtype=np.int64)
+    base = np.arange(G)
+    for o in range(d_out):
+        acc[:, o] = (xg[:, base, i0[o]] * vals[o, :, 0]).sum(axis=1) + (xg[:, base, i1[o]] * vals[o, :, 1]).sum(axis=1)
+    return acc.astype(np.int32)

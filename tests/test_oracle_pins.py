@@ -382,3 +382,74 @@ def test_gemv_packed_equals_forward():
     xq, amax = oracle.act_quant(synth.bits(x))
     y = oracle.gemv_packed(xq, amax, oracle.pack(weff, 6, 8), gamma, 128, 20, 6, 8)
     assert np.array_equal(y, oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax))
+
+
+# ---------------------------------------------------------------- 2:4 sparse operand (a8)
+def test_sparse24_hand_compressed_row():
+    kv = dict(_read_kv(os.path.join(GOLDEN, "sparse24_row.txt")))
+    d_out, d_in = int(kv["d_out"][0]), int(kv["d_in"][0])
+    weff = np.array([int(v) for v in kv["weff"]], np.int8).reshape(d_out, d_in)
+    buf = oracle.compress24(weff)
+    vrow, meta_off, total, KB, MB = oracle.sparse24_layout(d_out, d_in)
+    assert total == int(kv["total"][0]) and meta_off == int(kv["meta_off"][0]) and buf.size == total
+    assert [f"{b:02x}" for b in buf[:vrow]] == kv["values"]
+    assert np.all(buf[vrow:meta_off] == 0)
+    meta = buf[meta_off:]
+    assert [f"{b:02x}" for b in meta[:2]] == kv["meta"]
+    assert np.all(meta[2:] == 0x44)
+    assert np.array_equal(oracle.decompress24(buf, d_out, d_in), weff)
+
+
+def test_sparse24_every_group_pattern():
+    """All 81 ternary groups of four: two or fewer nonzeros compress to the
+    slots the definition names, anything more is rejected."""
+    import itertools
+    for grp in itertools.product((-1, 0, 1), repeat=4):
+        w = np.array(list(grp) + [0] * 12, np.int8).reshape(1, 16)
+        nz = [p for p in range(4) if grp[p] != 0]
+        if len(nz) > 2:
+            with pytest.raises(ValueError):
+                oracle.compress24(w)
+            continue
+        slots = sorted(nz + [p for p in range(4) if grp[p] == 0][: 2 - len(nz)])
+        buf = oracle.compress24(w)
+        assert buf[0] == np.uint8(grp[slots[0]] & 0xFF) and buf[1] == np.uint8(grp[slots[1]] & 0xFF)
+        _, meta_off, _, _, _ = oracle.sparse24_layout(1, 16)
+        assert buf[meta_off] & 0xF == slots[0] | (slots[1] << 2)
+        assert np.array_equal(oracle.decompress24(buf, 1, 16), w)
+
+
+def test_sparse24_block_placement():
+    """The selector of one group lands at the byte worked out by hand:
+    row 300, weights 388..391 of a 520 x 520 weight.  Row blocks of 128:
+    mb = 2, r = 44; weight blocks of 256: kb = 1, offset 132 -> half 1,
+    weight 4 of the half -> group 1 -> byte 0, high nibble.  KB = 3, so the
+    half starts at ((2 * 3 + 1) * 2 + 1) * 2048 = 30720 and the byte is
+    30720 + 44 * 16 = 31424 bytes into the selector plane."""
+    w = np.zeros((520, 520), np.int8)
+    w[300, 388 + 1] = 1
+    w[300, 388 + 3] = -1
+    buf = oracle.compress24(w)
+    vrow, meta_off, total, KB, MB = oracle.sparse24_layout(520, 520)
+    assert (vrow, KB, MB) == (260 + 12, 3, 6)
+    meta = buf[meta_off:]
+    assert meta[31424] == (0x4 | ((1 | 3 << 2) << 4))
+    meta2 = meta.copy()
+    meta2[31424] = 0x44
+    assert np.all(meta2 == 0x44)
+    assert buf[300 * vrow + 2 * 97] == 1 and buf[300 * vrow + 2 * 97 + 1] == 0xFF
+
+
+def test_sparse24_product_and_roundtrip_ragged():
+    """On 2:4 weights from the full weight step (ragged in both dimensions),
+    the product formed from kept values and selected activations equals the
+    dense product of W_eff, including the int8 extremes."""
+    w = synth.bits(synth.trimodal_weight(392, 784, seed=21))
+    weff, _, _ = oracle.effective_weight(w, 2, 4)
+    buf = oracle.compress24(weff)
+    assert np.array_equal(oracle.decompress24(buf, 392, 784), weff)
+    rng = np.random.default_rng(21)
+    xq = rng.integers(-128, 128, size=(19, 784)).astype(np.int8)
+    xq[0] = -128
+    xq[1] = 127
+    assert np.array_equal(oracle.forward_acc_sparse24(xq, buf, 392, 784), oracle.forward_acc(xq, weff))
