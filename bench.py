@@ -107,7 +107,8 @@ class Step:
         self.dX = {p.name: torch.empty(T, p.d_in, dtype=torch.float32, device=dev) for p in ls.projections}
         self.dW = {p.name: torch.empty(p.d_out, p.d_in, dtype=torch.float32, device=dev) for p in ls.projections}
         n_p, n_x = len(ls.projections), len(ls.inputs)
-        self.kernels_per_step = 2 * n_p + n_x + 3 * n_p
+        self.sparse24 = (N_KEEP, M_GROUP) == (2, 4)  # compress + sparse tensor-core forward
+        self.kernels_per_step = 2 * n_p + n_x + 3 * n_p + (n_p if self.sparse24 else 0)
 
     def run(self, stream, ev=None):
         """Enqueue one step.  With `ev` (dict name -> list), record event pairs per call."""
@@ -470,13 +471,16 @@ def main():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sbl", "reference"], default="sbl")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen2.5-3b")
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (0: the workload's default)")
     ap.add_argument("--mode", choices=["train", "decode", "prefill"], default="train")
     ap.add_argument("--layers", type=int, default=36, help="decode mode: distinct layer sets in the stack")
+    ap.add_argument("--nm", default="6:8", help="N:M of the mask (the sweep: 8:8, 6:8, 4:8, 2:8, 2:4)")
     args = ap.parse_args()
+    global N_KEEP, M_GROUP
+    N_KEEP, M_GROUP = (int(v) for v in args.nm.split(":"))
     if args.mode == "decode":
         run_decode(args)
         return
@@ -494,7 +498,9 @@ def main():
                           f", X ~ N(0,1)" + (f" with {outl:.1%} outlier channels x10" if outl else "") +
                           ", dY ~ N(0,1)",
               "tokens_per_step": T, "params": ls.params, "nm": f"{N_KEEP}:{M_GROUP}",
-              "l2": "per-step working set larger than L2, no flush", "parallelism": f"dp{args.gpus} replicas"}
+              "l2": "per-step working set larger than L2, no flush", "parallelism": f"dp{args.gpus} replicas",
+              "forward_kernel": ("2:4 compress + sparse int8 MMA (tcgen05.mma.sp)" if (N_KEEP, M_GROUP) == (2, 4)
+                                 else "dense int8 MMA (tcgen05.mma kind::i8)")}
 
     if args.impl == "reference":
         if rank != 0:
@@ -559,27 +565,56 @@ def main():
     per_call = {k: sum(a.elapsed_time(b) for a, b in v) / args.steps for k, v in ev.items()}
     launches = {k: len(v) // args.steps for k, v in ev.items()}
 
-    # ---- end to end through host buffers (pinned), copies inside the timed region
+    # ---- end to end through host buffers (pinned), copies inside the timed region.
+    # Every step copies its inputs (W, X, dY) host -> device and its results
+    # (y, dX, dW) device -> host.  Steps are pipelined on three streams over
+    # two device buffer sets: the upload of step i+1 and the download of
+    # step i-1 run while step i computes (PCIe is full duplex).
     h2d = sum(t.numel() * t.element_size() for d in (Wp, Xp, dYp) for t in d.values())
-    outs = [*step.Y.values(), *step.dX.values(), *step.dW.values()]
-    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-    d2h = sum(t.numel() * t.element_size() for t in outs)
+    sets = [(W, X, dY, step)]
+    if args.e2e_steps > 1:
+        with torch.cuda.stream(stream):
+            W2 = {k: torch.empty_like(v) for k, v in W.items()}
+            X2 = {k: torch.empty_like(v) for k, v in X.items()}
+            dY2 = {k: torch.empty_like(v) for k, v in dY.items()}
+            sets.append((W2, X2, dY2, Step(ls, T, W2, X2, dY2)))
+    outs_of = lambda st: [*st.Y.values(), *st.dX.values(), *st.dW.values()]  # noqa: E731
+    host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs_of(st)] for (_, _, _, st) in sets]
+    d2h = sum(t.numel() * t.element_size() for t in outs_of(step))
+    s_up, s_down = torch.cuda.Stream(), torch.cuda.Stream()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.e2e_steps):
-            for src, dst in ((Wp, W), (Xp, X), (dYp, dY)):
+    e0.record(s_up)
+    done_down = [None] * len(sets)
+    for i in range(args.e2e_steps):
+        b = i % len(sets)
+        Wd, Xd, dYd, st = sets[b]
+        if done_down[b] is not None:
+            s_up.wait_event(done_down[b])  # set b's previous step is computed and downloaded
+        with torch.cuda.stream(s_up):
+            for src, dst in ((Wp, Wd), (Xp, Xd), (dYp, dYd)):
                 for k in src:
                     dst[k].copy_(src[k], non_blocking=True)
-            step.run(stream)
-            for h, d in zip(host_out, outs):
+        up = torch.cuda.Event()
+        up.record(s_up)
+        stream.wait_event(up)
+        st.run(stream)
+        comp = torch.cuda.Event()
+        comp.record(stream)
+        s_down.wait_event(comp)
+        with torch.cuda.stream(s_down):
+            for h, d in zip(host_out[b], outs_of(st)):
                 h.copy_(d, non_blocking=True)
-    e1.record(stream)
-    stream.synchronize()
+        done_down[b] = torch.cuda.Event()
+        done_down[b].record(s_down)
+    s_down.wait_stream(stream)
+    s_down.wait_stream(s_up)
+    e1.record(s_down)
+    e1.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(1, args.e2e_steps), dist, "cuda")
     e2e_value = job_throughput(world, T, e2e_ms)
+    sbl.sbl_check(stream)
 
     # ---- roofline of the dominant call family and of the whole step
     pk = peaks()
@@ -616,7 +651,8 @@ def main():
             "vs_baseline": None, "dtype": "i8 fwd / bf16 bwd (fp32 accumulate)", "data": "synthetic",
             "config": config, "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms},
+                    "ms_per_step": e2e_ms, "steps": args.e2e_steps,
+                    "note": "pinned host buffers; uploads, steps and downloads pipelined on three streams"},
             "gpu_launches": step.kernels_per_step * args.steps,
             "per_call_ms_per_step": per_call, "clocks": clk.summary(),
         }))

@@ -171,6 +171,43 @@ sbl_status sbl_forward_packed(const int8_t* Xq, const float* amax, const uint8_t
                               float* Y, int32_t* acc, void* stream);
 
 /* ------------------------------------------------------------------------
+ * 2:4 weights on the sparse tensor core (tcgen05.mma.sp, kind::i8).
+ * [summary] 前置知识 / 半结构化 N:M 稀疏 (2:4 is the pattern sparse tensor
+ * cores accelerate) and 核心方法 (the mask is applied after quantisation,
+ * so a 2:4 W_eff is already in the structure the hardware takes).
+ *
+ * sbl_compress24 turns a 2:4 W_eff ([d_out, d_in] int8, at most two
+ * nonzeros in every group of four) into the compressed buffer the sparse
+ * forward reads:
+ *   values plane    d_out rows of ceil16(d_in / 2) bytes: the int8 values
+ *                   of each group's two slots, ascending position order;
+ *   selector plane  from the first 1024-byte boundary after the values: the
+ *                   4-bit selector i0 | i1 << 2 of every group, in blocks of
+ *                   128 rows x 256 weights (4096 bytes; block (mb, kb) at
+ *                   (mb * ceil(d_in/256) + kb) * 4096), each block two
+ *                   halves of 128 rows x 16 bytes, row r at 16 r, two groups
+ *                   per byte (low nibble = even group).  Rows are padded to a
+ *                   multiple of 256 and weights to a multiple of 256 with
+ *                   selector 0x4 (slots 0, 1) and zero values.
+ * Slots are the group's nonzero positions plus its lowest zero positions.
+ * A group with more than two nonzeros latches SBL_ERR_DEVICE_CHECK (its
+ * first two nonzeros are kept).
+ *   out        device buffer of at least sbl_compress24_bytes() bytes.
+ *
+ * sbl_forward_sparse24 computes exactly sbl_forward on the W_eff that was
+ * compressed, bit for bit (same int32 accumulators, same fp32 epilogue),
+ * with the multiply skipped for the two dropped weights of every group.
+ *   w24        sbl_compress24 output for this [d_out, d_in].
+ *   other arguments as sbl_forward.
+ * ---------------------------------------------------------------------- */
+size_t sbl_compress24_bytes(int d_out, int d_in);
+sbl_status sbl_compress24(const int8_t* W_eff, int d_out, int d_in, uint8_t* out,
+                          size_t out_bytes, void* stream);
+sbl_status sbl_forward_sparse24(const int8_t* Xq, const float* amax, const uint8_t* w24,
+                                const float* gamma, int T, int d_in, int d_out, float* Y,
+                                int32_t* acc, void* stream);
+
+/* ------------------------------------------------------------------------
  * Dual-STE backward on bf16 tensor cores (tcgen05, fp32 accumulation).
  * [summary] 前置知识 / STE and 核心方法 (masked weights receive the full
  * gradient), Algorithm 1 step (7):

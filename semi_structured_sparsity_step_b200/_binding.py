@@ -37,6 +37,9 @@ SIGNATURES = {
     "sbl_act_quant": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_forward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_forward_packed": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
+    "sbl_compress24_bytes": (_c_size, [_c_int, _c_int]),
+    "sbl_compress24": (_c_int, [_vp, _c_int, _c_int, _vp, _c_size, _vp]),
+    "sbl_forward_sparse24": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_backward_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
     "sbl_backward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp, _c_size, _vp]),
     "sbl_packed_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
@@ -151,6 +154,19 @@ def sbl_forward(Xq, amax, W_eff, gamma, T, d_in, d_out, Y, acc=None, stream=None
 def sbl_forward_packed(Xq, amax, packed, gamma, T, d_in, d_out, N, M, Y, acc=None, stream=None) -> None:
     _call("sbl_forward_packed", _ptr(Xq), _ptr(amax), _ptr(packed), _ptr(gamma), T, d_in, d_out, N, M, _ptr(Y),
           _ptr(acc), _stream(stream))
+
+
+def sbl_compress24_bytes(d_out, d_in) -> int:
+    return load().sbl_compress24_bytes(d_out, d_in)
+
+
+def sbl_compress24(W_eff, d_out, d_in, out, out_bytes, stream=None) -> None:
+    _call("sbl_compress24", _ptr(W_eff), d_out, d_in, _ptr(out), out_bytes, _stream(stream))
+
+
+def sbl_forward_sparse24(Xq, amax, w24, gamma, T, d_in, d_out, Y, acc=None, stream=None) -> None:
+    _call("sbl_forward_sparse24", _ptr(Xq), _ptr(amax), _ptr(w24), _ptr(gamma), T, d_in, d_out, _ptr(Y), _ptr(acc),
+          _stream(stream))
 
 
 def sbl_backward_workspace_bytes(T, d_in, d_out) -> int:

@@ -188,6 +188,41 @@ sbl_status sbl_forward_packed(const int8_t* Xq, const float* amax, const uint8_t
                                          static_cast<cudaStream_t>(stream), d->num_sms, d->err));
 }
 
+size_t sbl_compress24_bytes(int d_out, int d_in) {
+  if (check_dims(d_in, d_out) != SBL_OK) return 0;
+  return sparse24_bytes(d_out, d_in);
+}
+
+sbl_status sbl_compress24(const int8_t* W_eff, int d_out, int d_in, uint8_t* out, size_t out_bytes, void* stream) {
+  sbl_status st = check_dims(d_in, d_out);
+  if (st != SBL_OK) return st;
+  if (d_out == 0 || d_in == 0) return SBL_OK;
+  if (W_eff == nullptr || out == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(W_eff) || !aligned16(out)) return SBL_ERR_ALIGN;
+  if (out_bytes < sparse24_bytes(d_out, d_in)) return SBL_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  return from_cuda(launch_compress24(W_eff, d_out, d_in, out, static_cast<cudaStream_t>(stream), d->num_sms,
+                                     d->err));
+}
+
+sbl_status sbl_forward_sparse24(const int8_t* Xq, const float* amax, const uint8_t* w24, const float* gamma, int T,
+                                int d_in, int d_out, float* Y, int32_t* acc, void* stream) {
+  sbl_status st = check_dims(d_in, d_out);
+  if (st != SBL_OK) return st;
+  if (T < 0) return SBL_ERR_SHAPE;
+  if (T == 0 || d_out == 0) return SBL_OK;
+  if (Xq == nullptr || amax == nullptr || w24 == nullptr || gamma == nullptr || Y == nullptr)
+    return SBL_ERR_INVALID_ARG;
+  if (!aligned16(Xq) || !aligned16(amax) || !aligned16(w24) || !aligned16(Y) || !aligned16(acc) ||
+      (reinterpret_cast<uintptr_t>(gamma) & 3u) != 0)
+    return SBL_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  return from_cuda(launch_forward_sparse24(Xq, amax, w24, gamma, T, d_in, d_out, Y, acc,
+                                           static_cast<cudaStream_t>(stream), d->num_sms, d->err));
+}
+
 size_t sbl_backward_workspace_bytes(int T, int d_in, int d_out) {
   (void)T;
   (void)d_in;

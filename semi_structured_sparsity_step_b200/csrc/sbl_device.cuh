@@ -185,6 +185,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Descriptor of an unswizzled K-major tile whose rows are 16 bytes: the
+// 8-row core matrices are SBO bytes apart (128 when the rows are
+// contiguous); there is one core matrix along K, so LBO is unused.  This is
+// the source layout of tcgen05.cp.128x128b (128 rows x 16 bytes).
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t saddr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  return d;  // layout 0: no swizzle
+}
+
 // Instruction descriptor for kind::i8 (s8 x s8 -> s32) and kind::f16
 // (bf16 x bf16 -> f32):  bits 4-5 D format (1 f32, 2 s32), 7-9 A format,
 // 10-12 B format (i8: 1 = signed; f16 kind: 1 = bf16), 15 A MN-major,
@@ -282,6 +295,29 @@ __device__ __forceinline__ void umma_commit_multicast(uint64_t* bar, uint16_t ct
           smem_u32(bar)),
       "h"(cta_mask)
       : "memory");
+}
+
+// Sparse int8 MMA over the pair (tcgen05.mma.sp, kind::i8): A is the 2:4
+// compressed operand (32 bytes of kept values per row per instruction,
+// K = 64 logical), its selector metadata is read from TMEM at `e_tmem`.
+__device__ __forceinline__ void umma_sp_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t e_tmem, uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::i8 [%0], %1, %2, [%13], %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z),
+      "r"(z), "r"(e_tmem)
+      : "memory");
+}
+
+// Copy a 128-row x 16-byte shared-memory tile into 4 TMEM columns of lanes
+// 0-127, in each CTA of the pair from its own shared memory (issued by the
+// even CTA).  Ordered before the tcgen05.mma issued after it by the same
+// thread; tracked by the next tcgen05.commit.
+__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 }  // namespace pair

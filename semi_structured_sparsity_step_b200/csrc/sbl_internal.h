@@ -34,6 +34,9 @@ cudaError_t launch_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* 
 // bytes), box [box_rows, box_inner], no swizzle; out-of-range elements read 0.
 bool make_tmap_u32(CUtensorMap* m, const void* base, unsigned long long inner, unsigned long long rows,
                    unsigned long long row_bytes, unsigned box_inner, unsigned box_rows);
+// Same for a uint8 matrix, with the 128-byte swizzle or none.
+bool make_tmap_u8(CUtensorMap* m, const void* base, unsigned long long inner, unsigned long long rows,
+                  unsigned long long row_bytes, unsigned box_inner, unsigned box_rows, bool swizzle128);
 extern int g_gemm_variant;
 cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
                            int d_in, int d_out, float* Y, int32_t* acc, cudaStream_t stream, int num_sms,
@@ -44,6 +47,16 @@ cudaError_t launch_forward_packed(const int8_t* Xq, const float* amax, const uin
 cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf16, const float* gamma, int T,
                             int d_in, int d_out, float* dX, float* dW, int accumulate_dW, cudaStream_t stream,
                             int num_sms, uint32_t* err);
+
+// ---- 2:4 compressed weight and the sparse tensor-core forward (gemm_sp24.cu)
+size_t sparse24_values_row_bytes(int d_in);
+size_t sparse24_meta_offset(int d_out, int d_in);
+size_t sparse24_bytes(int d_out, int d_in);
+cudaError_t launch_compress24(const int8_t* W_eff, int d_out, int d_in, uint8_t* out, cudaStream_t stream,
+                              int num_sms, uint32_t* err);
+cudaError_t launch_forward_sparse24(const int8_t* Xq, const float* amax, const uint8_t* w24, const float* gamma,
+                                   int T, int d_in, int d_out, float* Y, int32_t* acc, cudaStream_t stream,
+                                   int num_sms, uint32_t* err);
 
 // ---- packed format (pack_gemv.cu)
 size_t packed_codes_row_bytes(int d_in, int N, int M);
