@@ -205,14 +205,20 @@ def backward_dw(dy_bits: np.ndarray, x_bits: np.ndarray) -> np.ndarray:
 # (a9) packed inference format: 2-bit ternary codes + N:M index
 # [article] 7.1 推理优化技巧 (pre-compute and cache the sparse format; bit
 # operations for ternary products); [summary] 核心方法 (the deployed ternary
-# weights are N:M-structured).
+# weights are N:M-structured).  The pages fix only "2-bit ternary codes plus
+# an N:M index"; the bit layout below is this library's.
 #
 # Per weight row, two planes, each padded to a multiple of 16 bytes:
-#   codes plane: for every group of M, the codes of its N slots in ascending
-#     position order, 2 bits each (00 -> 0, 01 -> +1, 11 -> -1), written as
-#     a little-endian bit stream (code i of group g at bit 2*(g*N + i));
 #   index plane: for every group, an M-bit slot mask (bit p = position p is a
-#     slot), little-endian bit stream (group g at bit g*M).
+#     slot), little-endian bit stream (group g at bit g*M);
+#   codes plane: the row is cut into chunks of 8 consecutive positions (one
+#     group when M = 8, two when M = 4).  A chunk has K = 8N/M slots s_0 <
+#     ... < s_(K-1) (its groups' slots in ascending position order) and a
+#     field of 2K bits; chunk c's field starts at bit 2K*c of a little-endian
+#     bit stream.  With H = ceil(K/2), the code of slot s_q (q < H) sits at
+#     field bits 4q, 4q+1 and the code of slot s_(H+q) at bits 4q+2, 4q+3.
+#   Code of a value: +1 -> 00, -1 -> 01, 0 -> 10 (bit 0 = negative, bit 1 =
+#     zero); 11 is never written.
 # Slots are all nonzero positions of the group plus, if there are fewer
 # than N, the lowest-index zero positions.  The buffer holds all code rows
 # first, then all index rows.
@@ -243,8 +249,21 @@ def _get_bits(buf, bitpos: int, nbits: int) -> int:
     return v
 
 
-_CODE = {0: 0b00, 1: 0b01, -1: 0b11}
-_VALUE = {0b00: 0, 0b01: 1, 0b11: -1}
+_CODE = {1: 0b00, -1: 0b01, 0: 0b10}
+_VALUE = {0b00: 1, 0b01: -1, 0b10: 0}
+
+
+def _slot_bit(i: int, K: int) -> int:
+    """Bit offset, inside its chunk's field, of the code of slot i."""
+    H = (K + 1) // 2
+    return 4 * i if i < H else 4 * (i - H) + 2
+
+
+def _group_slots(grp, N: int):
+    """The slots of one group: nonzero positions, then lowest zero positions."""
+    nz = [p for p in range(len(grp)) if grp[p] != 0]
+    zeros = [p for p in range(len(grp)) if grp[p] == 0]
+    return sorted(nz + zeros[: max(0, N - len(nz))])
 
 
 def pack(weff: np.ndarray, N: int, M: int) -> np.ndarray:
@@ -252,23 +271,26 @@ def pack(weff: np.ndarray, N: int, M: int) -> np.ndarray:
     d_out, d_in = weff.shape
     crow, irow, total = packed_layout(d_out, d_in, N, M)
     G = d_in // M
+    K = 8 * N // M
     out = bytearray(total)
     for o in range(d_out):
         codes = bytearray(crow)
         index = bytearray(irow)
-        for g in range(G):
-            grp = [int(v) for v in weff[o, g * M:(g + 1) * M]]
-            nz = [p for p in range(M) if grp[p] != 0]
-            if len(nz) > N:
-                raise ValueError(f"row {o} group {g}: {len(nz)} nonzeros > N={N}")
-            zeros = [p for p in range(M) if grp[p] == 0]
-            slots = sorted(nz + zeros[: N - len(nz)])
-            _put_bits(index, g * M, sum(1 << p for p in slots), M)
-            for i, p in enumerate(slots):
-                _put_bits(codes, 2 * (g * N + i), _CODE[grp[p]], 2)
+        for c in range(d_in // 8):
+            chunk_slots = []                      # positions within the chunk
+            for g in range(c * 8 // M, (c + 1) * 8 // M):
+                grp = [int(v) for v in weff[o, g * M:(g + 1) * M]]
+                if sum(v != 0 for v in grp) > N:
+                    raise ValueError(f"row {o} group {g}: more than N={N} nonzeros")
+                slots = _group_slots(grp, N)
+                _put_bits(index, g * M, sum(1 << p for p in slots), M)
+                chunk_slots += [g * M + p - 8 * c for p in slots]
+            for i, p in enumerate(chunk_slots):
+                _put_bits(codes, 2 * K * c + _slot_bit(i, K), _CODE[int(weff[o, 8 * c + p])], 2)
         out[o * crow:(o + 1) * crow] = codes
         base = d_out * crow
         out[base + o * irow: base + (o + 1) * irow] = index
+    assert G * M == d_in
     return np.frombuffer(bytes(out), dtype=np.uint8).copy()
 
 
@@ -276,23 +298,26 @@ def unpack(packed: np.ndarray, d_out: int, d_in: int, N: int, M: int) -> np.ndar
     """Inverse of :func:`pack` (raises on an invalid code or slot count)."""
     crow, irow, total = packed_layout(d_out, d_in, N, M)
     assert packed.size == total
-    G = d_in // M
+    K = 8 * N // M
     buf = packed.tobytes()
     w = np.zeros((d_out, d_in), dtype=np.int8)
     base = d_out * crow
     for o in range(d_out):
         codes = buf[o * crow:(o + 1) * crow]
         index = buf[base + o * irow: base + (o + 1) * irow]
-        for g in range(G):
-            m = _get_bits(index, g * M, M)
-            slots = [p for p in range(M) if (m >> p) & 1]
-            if len(slots) != N:
-                raise ValueError(f"row {o} group {g}: {len(slots)} slots != N={N}")
-            for i, p in enumerate(slots):
-                c = _get_bits(codes, 2 * (g * N + i), 2)
-                if c not in _VALUE:
-                    raise ValueError(f"row {o} group {g}: invalid code {c:#b}")
-                w[o, g * M + p] = _VALUE[c]
+        for c in range(d_in // 8):
+            chunk_slots = []
+            for g in range(c * 8 // M, (c + 1) * 8 // M):
+                m = _get_bits(index, g * M, M)
+                slots = [p for p in range(M) if (m >> p) & 1]
+                if len(slots) != N:
+                    raise ValueError(f"row {o} group {g}: {len(slots)} slots != N={N}")
+                chunk_slots += [g * M + p - 8 * c for p in slots]
+            for i, p in enumerate(chunk_slots):
+                code = _get_bits(codes, 2 * K * c + _slot_bit(i, K), 2)
+                if code not in _VALUE:
+                    raise ValueError(f"row {o} chunk {c}: invalid code {code:#b}")
+                w[o, 8 * c + p] = _VALUE[code]
     return w
 
 

@@ -342,7 +342,7 @@ def test_pack_hand_packed_rows():
             cases.append({"N": int(vals[0]), "M": int(vals[1])})
         else:
             cases[-1][key] = vals
-    assert len(cases) == 2
+    assert len(cases) == 4
     for c in cases:
         N, M = c["N"], c["M"]
         weff = np.array([int(v) for v in c["weff"]], np.int8).reshape(1, -1)
@@ -358,7 +358,7 @@ def test_pack_hand_packed_rows():
         assert np.array_equal(oracle.unpack(p, 1, weff.shape[1], N, M), weff)
 
 
-@pytest.mark.parametrize("N,M", [(6, 8), (2, 4), (8, 8), (2, 8)])
+@pytest.mark.parametrize("N,M", [(6, 8), (2, 4), (8, 8), (2, 8), (3, 8), (5, 8), (1, 4), (3, 4), (4, 4)])
 def test_pack_roundtrip(N, M):
     w = synth.bits(synth.trimodal_weight(6, 96, seed=14))
     weff, _, _ = oracle.effective_weight(w, N, M)
