@@ -30,6 +30,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "packed_decode.cuh"
 #include "sbl_device.cuh"
 #include "sbl_internal.h"
 
@@ -338,7 +339,7 @@ struct Cfg2 {
   static constexpr int EPI_WARP_FLOATS = 32 * 33;
   static constexpr int EPI_BYTES = 4 * EPI_WARP_FLOATS * 4;
   // Packed B (KP > 0): per-lane replicated decode tables after the barriers.
-  static constexpr int LUT_BYTES = KP > 0 ? (64 + 256) * 32 * 4 : 0;
+  static constexpr int LUT_BYTES = KP > 0 ? 256 * 32 * 8 + 256 * 8 : 0;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256 + LUT_BYTES;
   static constexpr int THREADS = KP > 0 ? 448 : 192;  // packed: + 8 decoder warps
   static constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -353,16 +354,15 @@ struct PackedB {
   int rows;              // d_out
 };
 
-__device__ __forceinline__ uint32_t packed_code_byte(uint32_t code) {
-  return code == 1u ? 0x01u : (code == 3u ? 0xFFu : 0u);
-}
-
 // Decodes half `hf` (chunks 8 hf .. 8 hf + 7, 64 weights) of K block `kb`
 // of weight row `row` from the packed planes into row `r` of a 128 x
 // 128-byte int8 B tile with the 128-byte swizzle (16-byte unit c of row r
 // stored at unit c ^ (r % 8)), the layout a TMA load of W_eff would produce.
-// Chunks past d_in/8 and rows past d_out decode to zeros.  Tables are
-// replicated per lane (entry e of copy l at word e * 32 + l).
+// Rows past d_out and chunks past d_in/8 load as zero words; what they decode
+// to is never used (their outputs are not stored, and the matching
+// activations are zero-filled by TMA).  The chunk decoder is the byte-permute
+// one of packed_decode.cuh; the scatter-selector table is replicated per
+// lane (the entry of mask m for lane l at byte m * 256 + l * 8).
 template <int KP>
 struct PackedHalf {
   uint32_t w[(KP + 1) / 2 + 1];  // 8 chunks x 2KP bits = 2KP bytes (+1 word of zeros)
@@ -398,7 +398,7 @@ __device__ __forceinline__ void load_packed_half(PackedHalf<KP>& ph, const Packe
 
 template <int KP>
 __device__ __forceinline__ void expand_packed_half(const PackedHalf<KP>& ph, int hf, uint8_t* tile, int r,
-                                                   const uint32_t* s_code, const uint32_t* s_sel, int lane) {
+                                                   const uint8_t* sel_bytes, uint32_t lane8) {
   const uint32_t* w = ph.w;
   const uint2 m = ph.m;
 #pragma unroll
@@ -408,19 +408,14 @@ __device__ __forceinline__ void expand_packed_half(const PackedHalf<KP>& ph, int
     for (int h = 0; h < 2; ++h) {
       const int j = 2 * c + h;  // chunk within the half
       const int bit = 2 * KP * j;
-      const uint32_t v = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31);
-      const uint32_t codes = (2 * KP == 32) ? v : (v & ((1u << (2 * KP)) - 1u));
-      const uint32_t mask = ((j < 4 ? m.x : m.y) >> (8 * (j & 3))) & 0xFFu;
-      uint32_t lo = s_code[((codes & 63u) << 5) + lane], hi = 0u;
-      if constexpr (KP > 3) {
-        const uint32_t t1 = s_code[(((codes >> 6) & 63u) << 5) + lane];
-        lo |= t1 << 24;
-        hi = t1 >> 8;
-        if constexpr (KP > 6) hi |= s_code[(((codes >> 12) & 63u) << 5) + lane] << 16;
-      }
-      const uint32_t sel = s_sel[(mask << 5) + lane];
-      out[2 * h] = __byte_perm(lo, hi, sel & 0xFFFFu);
-      out[2 * h + 1] = __byte_perm(lo, hi, sel >> 16);
+      const int wi = bit >> 5, sh = bit & 31;
+      const uint32_t v = sh == 0 ? w[wi] : __funnelshift_r(w[wi], w[wi + 1], sh);
+      uint32_t lo, hi;
+      ChunkCodes<KP>::decode(v, lo, hi);
+      const uint32_t amsel = 0x5504u | (static_cast<uint32_t>(j & 3) << 4);
+      const uint2 sel = *reinterpret_cast<const uint2*>(sel_bytes + prmt(j < 4 ? m.x : m.y, lane8, amsel));
+      out[2 * h] = prmt(lo, hi, sel.x);
+      out[2 * h + 1] = prmt(lo, hi, sel.y);
     }
     const int unit = 4 * hf + c;  // 16-byte unit within the 128-byte row
     *reinterpret_cast<uint4*>(tile + r * 128 + ((unit ^ (r & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
@@ -441,8 +436,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint32_t* s_code = reinterpret_cast<uint32_t*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES + 256);  // KP > 0
-  uint32_t* s_sel = s_code + 64 * 32;
+  uint8_t* sel_bytes = smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES + 256;  // KP > 0: [256][32] uint2
+  uint2* sel_one = reinterpret_cast<uint2*>(sel_bytes + 256 * 32 * 8);        // KP > 0: [256] uint2
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -454,21 +449,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
   const uint32_t peer_abort = pair::map_to(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
 
   if constexpr (KP > 0) {
-    for (int i = threadIdx.x; i < 64 * 32; i += blockDim.x) {
-      const uint32_t c = static_cast<uint32_t>(i) >> 5;
-      s_code[i] = packed_code_byte(c & 3u) | (packed_code_byte((c >> 2) & 3u) << 8) |
-                  (packed_code_byte((c >> 4) & 3u) << 16);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+      uint32_t s0, s1;
+      scatter_selectors(static_cast<uint32_t>(i), KP, s0, s1);
+      sel_one[i] = make_uint2(s0, s1);
     }
-    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-      const uint32_t c = static_cast<uint32_t>(i) >> 5;
-      uint32_t sel = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t nib = ((c >> q) & 1u) ? static_cast<uint32_t>(__popc(c & ((1u << q) - 1u))) : 7u;
-        sel |= nib << (4 * q);
-      }
-      s_sel[i] = sel;
-    }
+    __syncthreads();
+    uint2* tab = reinterpret_cast<uint2*>(sel_bytes);
+    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) tab[i] = sel_one[i >> 5];
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -631,7 +619,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
           break;
         }
         uint8_t* sb = smem + s * C::STAGE_BYTES + C::A_BYTES;
-        expand_packed_half<KP>(cur, hf, sb, r, s_code, s_sel, lane);
+        expand_packed_half<KP>(cur, hf, sb, r, sel_bytes, static_cast<uint32_t>(lane) * 8u);
         // make the generic-proxy stores visible to the tensor core (async proxy)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();

@@ -2,8 +2,11 @@
 //
 // Format (per weight row, two planes each padded to 16 bytes; all code rows
 // first, then all index rows):
-//   codes plane: the N slot codes of every group of M in ascending position
-//     order, 2 bits each (00 = 0, 01 = +1, 11 = -1), little-endian bit stream;
+//   codes plane: per chunk of 8 positions (one group at M = 8, two at M = 4;
+//     K = 8N/M slots s_0 < ... < s_(K-1), H = ceil(K/2)) a field of 2K bits
+//     at bit 2K * chunk of a little-endian bit stream; the code of s_q
+//     (q < H) sits at field bits 4q..4q+1, the code of s_(H+q) at 4q+2..4q+3;
+//     codes +1 = 00, -1 = 01, 0 = 10 (packed_decode.cuh decodes them);
 //   index plane: the M-bit slot mask of every group, little-endian bit stream.
 //   Slots = the group's nonzero positions plus, if fewer than N, its lowest
 //   zero positions.
@@ -21,6 +24,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "packed_decode.cuh"
 #include "sbl_device.cuh"
 #include "sbl_internal.h"
 
@@ -55,9 +59,11 @@ __global__ void pack_kernel(const int8_t* __restrict__ W, int d_out, int d_in, i
   const int8_t* wr = W + static_cast<size_t>(row) * d_in;
 
   unsigned __int128 cbuf = 0;  // code bits of this thread's chunks (<= 8 * 16 bits)
-  int cnt = 0;
+  const int K = gpc * N;        // slots per chunk
+  const int H = (K + 1) / 2;
   bool bad = false;
   for (int ch = c0; ch < c1; ++ch) {
+    int slot = 0;  // slot index within the chunk
     const uint2 v = *reinterpret_cast<const uint2*>(wr + 8 * ch);
     const uint32_t b[2] = {v.x, v.y};
     uint32_t mask8 = 0;
@@ -96,16 +102,17 @@ __global__ void pack_kernel(const int8_t* __restrict__ W, int d_out, int d_in, i
         if (!((slots >> p) & 1u)) continue;
         const int pos = g * M + p;
         const int8_t q = static_cast<int8_t>((b[pos >> 2] >> (8 * (pos & 3))) & 0xFFu);
-        const uint32_t code = q > 0 ? 1u : (q < 0 ? 3u : 0u);
-        cbuf |= static_cast<unsigned __int128>(code) << cnt;
-        cnt += 2;
+        const uint32_t code = q > 0 ? 0u : (q < 0 ? 1u : 2u);  // +1 00, -1 01, 0 10
+        const int fbit = slot < H ? 4 * slot : 4 * (slot - H) + 2;
+        cbuf |= static_cast<unsigned __int128>(code) << ((ch - c0) * 2 * K + fbit);
+        ++slot;
       }
     }
     index[ch] = static_cast<uint8_t>(mask8);
   }
   // code bits of chunk c0 start at bit c0 * cbits, a multiple of 8 (c0 % 8 == 0).
   const size_t byte0 = static_cast<size_t>(c0) * cbits / 8;
-  const int nbytes = (cnt + 7) / 8;
+  const int nbytes = ((c1 - c0) * 2 * K + 7) / 8;
   for (int k = 0; k < nbytes; ++k) codes[byte0 + k] = static_cast<uint8_t>(cbuf >> (8 * k));
   if (bad) latch_error(err, kErrDeviceCheck);
 }
@@ -113,28 +120,40 @@ __global__ void pack_kernel(const int8_t* __restrict__ W, int d_out, int d_in, i
 // ------------------------------------------------------------------- GEMV
 // Decode GEMV on int8 tensor cores (mma.sync m16n8k32, s8 x s8 -> s32).
 //
-// A warp computes 16 weight rows x all tokens (up to 16) over a K slice.  The
-// order of the K sum is free, so the 32 k positions of each mma are chosen
-// to suit the format: within a block of 32 chunks (256 weights of a row),
-// lane (g, t) (g = lane / 4, t = lane % 4) owns the 8 consecutive chunks
-// 8t .. 8t+7, i.e. one aligned run of 2K code bytes and 8 index bytes per
-// row; mma number j of the block takes chunk 8t + j from every t.  A chunk
-// decodes to 8 int8 weights: positions 0-3 go to k = 4t..4t+3 (A registers
-// a0 / a1 for rows g / g+8) and positions 4-7 to k = 16+4t..16+4t+3 (a2 /
-// a3).  The B fragment of token n = g is then the 8 int8 activations of the
-// same chunk (b0 = positions 0-3, b1 = 4-7): one 8-byte load.  Decoding a
-// chunk: its 2K code bits (K = 8N/M slots), two table lookups (4 codes ->
-// 4 int8 each) and two __byte_perm with selectors looked up from the 8-bit
-// slot mask.  Warps of a block that share 16 rows split K and add their
-// int32 partial sums through shared memory; the result is scaled by
-// fp32(gamma * fp32(amax_b / 127)) per token.
+// A work unit is 16 (or 8) weight rows of one problem over its whole K; a
+// block's 8 consumer warps split every K tile of 256 chunks, 32 chunks each,
+// and add their int32 partial sums through shared memory at the end of the
+// unit.  The order of the K sum is free, so the 32 k positions of each mma
+// are chosen to suit the format: lane (g, t) (g = lane / 4, t = lane % 4)
+// owns the 8 consecutive chunks 8t .. 8t+7 of its warp's 32, i.e. one
+// aligned run of 2K code bytes and 8 index bytes per row; mma j of the tile
+// takes chunk 8t + j from every t.  A chunk decodes to 8 int8 weights:
+// positions 0-3 go to k = 4t..4t+3 (A registers a0 / a1 for rows g / g+8)
+// and positions 4-7 to k = 16+4t..16+4t+3 (a2 / a3); the B fragment of token
+// n = g is then the 8 activations of the same chunk (b0 = positions 0-3,
+// b1 = 4-7).  Decoding one chunk (packed_decode.cuh) is two byte permutes
+// against constants (slot codes -> int8 values), one permute that builds
+// the selector-table address from the slot-mask byte, one 8-byte table load
+// and two permutes that move the slot values to their positions.
+//
+// Problems whose K is at least twice the shortest K of the launch use 8-row
+// units (rows g only; a1 = a3 = 0), and units are numbered heaviest problem
+// first, so that the persistent blocks' static round-robin over units stays
+// balanced.  At the end of a unit each consumer warp adds its int32 partial
+// sums into a double-buffered shared accumulator (shared-memory atomics,
+// exact and order-free) and moves on; an epilogue warp scales the finished
+// sums by fp32(gamma * fp32(amax_b / 127)) and stores them, so no consumer
+// ever waits on an output store.  The kernel is launched with programmatic
+// dependent launch: the selector table is built and the weight tiles start
+// streaming while the previous kernel on the stream finishes; activations,
+// scales and outputs are touched only after griddepcontrol.wait.
 constexpr int kGemvMaxGroup = 16;
 
 struct alignas(64) GemvGroup {
-  CUtensorMap tm_codes[kGemvMaxGroup];  // codes plane as uint32 [d_out, crow / 4]
-  CUtensorMap tm_index[kGemvMaxGroup];  // index plane as uint32 [d_out, irow / 4]
+  CUtensorMap tm_codes[kGemvMaxGroup];  // codes plane as uint32 [d_out, crow / 4], box rows = unit rows
+  CUtensorMap tm_index[kGemvMaxGroup];  // index plane as uint32 [d_out, irow / 4], box rows = unit rows
   GemvProblemDev p[kGemvMaxGroup];
-  int block_start[kGemvMaxGroup + 1];   // first work item (16-row group) of each problem
+  int unit_start[kGemvMaxGroup + 1];    // first work unit of each problem
   int count, batch;
 };
 
@@ -147,132 +166,224 @@ __device__ __forceinline__ void mma_s8_16x8x32(int (&d)[4], uint32_t a0, uint32_
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Code bits of chunk j (0..7) of a run of 8 chunks held in words w[] (2K bits each).
+// Code field of chunk j (0..7) of a run of 8 chunks held in words w[] (2K bits each).
 template <int K>
-__device__ __forceinline__ uint32_t chunk_codes(const uint32_t (&w)[5], int j) {
+__device__ __forceinline__ uint32_t chunk_field(const uint32_t (&w)[5], int j) {
   const int bit = 2 * K * j;
   const int wi = bit >> 5, sh = bit & 31;
-  const uint32_t v = __funnelshift_r(w[wi], w[wi + 1], sh);
-  return (2 * K == 32) ? v : (v & ((1u << (2 * K)) - 1u));
+  return sh == 0 ? w[wi] : __funnelshift_r(w[wi], w[wi + 1], sh);
 }
 
-// Lookup tables, replicated once per lane: entry e of copy l sits at word
-// e * 32 + l, so lane l always reads bank l and lookups with 32 different
-// indices never conflict.
-//   code table (64 entries): 3 codes (6 bits) -> 3 int8 values (bytes 0-2);
-//   selector table (256 entries): slot mask -> two __byte_perm selectors
-//     (low 16 bits: positions 0-3, high 16 bits: positions 4-7) that move
-//     slot value i to the position of the i-th set bit and a zero byte
-//     (byte 7 of the value pair, always 0) elsewhere.
-constexpr int kCodeEntries = 64;
+// Scatter-selector table, replicated once per lane: the entry of slot mask
+// m for lane l is the uint2 at byte m * 256 + l * 8, so lane l always reads
+// banks 2l, 2l+1 and a warp's 32 lookups never conflict.
 constexpr int kSelEntries = 256;
+constexpr int kSelTableBytes = kSelEntries * 32 * 8;
 
-__device__ __forceinline__ uint32_t code_byte(uint32_t code) {
-  return code == 1u ? 0x01u : (code == 3u ? 0xFFu : 0u);
-}
-
-// Tile of one work item: 16 weight rows x 256 chunks (2048 weights) of K.
-// Codes: 16 rows x 64K bytes, index: 16 rows x 256 bytes, both loaded by 2-D
-// TMA (uint32 elements, no swizzle) into one stage of a shared-memory ring.
-constexpr int kGemvStages = 4;
+// Tile of one stage: up to 16 weight rows x 256 chunks (2048 weights) of K.
+// Codes: rows x 64K bytes, index: rows x 256 bytes, both loaded by 2-D TMA
+// (uint32 elements, no swizzle) into one stage of a shared-memory ring.
 constexpr int kTileChunks = 256;
-constexpr int kGemvThreads = 288;  // 8 consumer warps + 1 producer warp
+constexpr int kGemvThreads = 320;  // 8 consumer warps + 1 producer warp + 1 epilogue warp
 
 template <int K>
 struct GemvTile {
   static constexpr int CODE_ROW = kTileChunks * 2 * K / 8;  // bytes per row
   static constexpr int INDEX_ROW = kTileChunks;              // bytes per row
   static constexpr int BYTES = 16 * (CODE_ROW + INDEX_ROW);
+  // as many stages as still fit two blocks per SM
+  static constexpr int STAGES = K <= 6 ? 4 : 3;
+  static constexpr int SMEM = STAGES * BYTES + kSelTableBytes + kSelEntries * 8 + 128;
 };
 
-// Persistent: each block walks the work items (16 rows of one problem) with
-// stride gridDim.x and, within an item, its K tiles.  Warp 8 (one thread)
-// issues the TMA loads kGemvStages tiles ahead; warps 0-7 each decode 32
-// chunks (a 32 x 16 weight slab) of every tile into mma.sync fragments
-// (k order as described above), keep the int32 sums of the item in
-// registers, and after its last K tile add their partial sums through
-// shared memory and write the scaled outputs.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+// One K tile of one consumer warp: decode this lane's 8 chunks of row g
+// (and g + 8 when TWO) from the stage and multiply them into acc.
+template <int K, int NT, bool TWO>
+__device__ __forceinline__ void gemv_tile(int (&acc)[2][NT][4], const uint8_t* st, const uint8_t* sel_bytes,
+                                          const uint4 (&xv)[NT][4], int warp, int g, int t, uint32_t lane8) {
+  using Tl = GemvTile<K>;
+  using CC = ChunkCodes<K>;
+  const int coff = (warp * 32 + 8 * t) * 2 * K / 8;
+  uint32_t wa[5] = {0u, 0u, 0u, 0u, 0u}, wb[5] = {0u, 0u, 0u, 0u, 0u};
+  if constexpr ((K & 1) == 0) {
+#pragma unroll
+    for (int i = 0; i < K / 2; ++i) {
+      wa[i] = *reinterpret_cast<const uint32_t*>(st + g * Tl::CODE_ROW + coff + 4 * i);
+      if constexpr (TWO) wb[i] = *reinterpret_cast<const uint32_t*>(st + (g + 8) * Tl::CODE_ROW + coff + 4 * i);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      wa[i >> 1] |= static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(st + g * Tl::CODE_ROW + coff + 2 * i))
+                    << (16 * (i & 1));
+      if constexpr (TWO)
+        wb[i >> 1] |= static_cast<uint32_t>(
+                          *reinterpret_cast<const uint16_t*>(st + (g + 8) * Tl::CODE_ROW + coff + 2 * i))
+                      << (16 * (i & 1));
+    }
+  }
+  const uint8_t* ib = st + 16 * Tl::CODE_ROW;
+  const uint2 ma = *reinterpret_cast<const uint2*>(ib + g * Tl::INDEX_ROW + warp * 32 + 8 * t);
+  uint2 mb = make_uint2(0u, 0u);
+  if constexpr (TWO) mb = *reinterpret_cast<const uint2*>(ib + (g + 8) * Tl::INDEX_ROW + warp * 32 + 8 * t);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    // mask byte j -> byte 1 of the table offset, lane * 8 in byte 0
+    const uint32_t amsel = 0x5504u | (static_cast<uint32_t>(j & 3) << 4);
+    uint32_t lo, hi;
+    CC::decode(chunk_field<K>(wa, j), lo, hi);
+    const uint2 sa = *reinterpret_cast<const uint2*>(sel_bytes + prmt(j < 4 ? ma.x : ma.y, lane8, amsel));
+    const uint32_t a0 = prmt(lo, hi, sa.x), a2 = prmt(lo, hi, sa.y);
+    uint32_t a1 = 0u, a3 = 0u;
+    if constexpr (TWO) {
+      CC::decode(chunk_field<K>(wb, j), lo, hi);
+      const uint2 sb = *reinterpret_cast<const uint2*>(sel_bytes + prmt(j < 4 ? mb.x : mb.y, lane8, amsel));
+      a1 = prmt(lo, hi, sb.x);
+      a3 = prmt(lo, hi, sb.y);
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const uint4 x = xv[n][j >> 1];
+      mma_s8_16x8x32(acc[j & 1][n], a0, a1, a2, a3, (j & 1) ? x.z : x.x, (j & 1) ? x.w : x.y);
+    }
+  }
+}
+
+// Persistent: each block walks the work units with stride gridDim.x and,
+// within a unit, its K tiles.  Warp 8 (one thread) issues the TMA loads
+// Tl::STAGES tiles ahead; warps 0-7 decode and multiply; warp 9 finishes
+// the units (scale and store).
 template <int K, int NT>
 __global__ void __launch_bounds__(kGemvThreads, 2)
     gemv_packed_kernel(const __grid_constant__ GemvGroup grp, uint32_t* err) {
   using Tl = GemvTile<K>;
+  using CC = ChunkCodes<K>;
+  // Every shared pointer below is derived from gsm_raw by pointer arithmetic
+  // (no integer casts), so the compiler keeps them in the shared window and
+  // emits shared-memory loads with 32-bit addresses.
   extern __shared__ __align__(128) uint8_t gsm_raw[];
-  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 127) & ~uintptr_t(127));
-  uint32_t* s_code = reinterpret_cast<uint32_t*>(ring + kGemvStages * Tl::BYTES);  // [64][32]
-  uint32_t* s_sel = s_code + kCodeEntries * 32;                                      // [256][32]
-  __shared__ int s_part[8][16][16];
-  __shared__ __align__(8) uint64_t s_full[kGemvStages], s_empty[kGemvStages];
+  uint8_t* sel_bytes = gsm_raw;                                                 // [256][32] uint2
+  uint2* sel_one = reinterpret_cast<uint2*>(gsm_raw + kSelTableBytes);          // [256] uint2
+  const uint32_t ring_off = kSelTableBytes + kSelEntries * 8;
+  uint8_t* ring = gsm_raw + ring_off + ((128u - ((smem_u32(gsm_raw) + ring_off) & 127u)) & 127u);
+  __shared__ int s_acc[2][16][16];                  // unit sums [buffer][row][token]
+  __shared__ float s_scale[kGemvMaxGroup][16];      // gamma * amax_tok / 127 per problem
+  __shared__ __align__(8) uint64_t s_full[4], s_empty[4];
+  __shared__ __align__(8) uint64_t s_accf[2], s_acce[2];
   __shared__ int s_abort;
 
-  for (int i = threadIdx.x; i < kCodeEntries * 32; i += blockDim.x) {
-    const uint32_t c = static_cast<uint32_t>(i) >> 5;
-    s_code[i] = code_byte(c & 3u) | (code_byte((c >> 2) & 3u) << 8) | (code_byte((c >> 4) & 3u) << 16);
-  }
-  for (int i = threadIdx.x; i < kSelEntries * 32; i += blockDim.x) {
-    const uint32_t c = static_cast<uint32_t>(i) >> 5;
-    uint32_t sel = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const uint32_t nib = ((c >> q) & 1u) ? static_cast<uint32_t>(__popc(c & ((1u << q) - 1u))) : 7u;
-      sel |= nib << (4 * q);
-    }
-    s_sel[i] = sel;
-  }
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kGemvStages; ++i) {
+    for (int i = 0; i < Tl::STAGES; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 8);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_accf[b], 8);
+      mbar_init(&s_acce[b], 1);
     }
     s_abort = 0;
     fence_mbar_init();
   }
-  __syncthreads();
+  __syncthreads();  // barriers initialised
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total = grp.block_start[grp.count];
+  if (warp != 8) {
+    // Warps 0-7 and 9 build the selector table and clear the accumulators
+    // while the producer (warp 8) already streams the first tiles; named
+    // barrier 1 joins only these 288 threads.
+    const int tid = warp == 9 ? 256 + lane : static_cast<int>(threadIdx.x);
+    for (int i = tid; i < kSelEntries; i += 288) {
+      uint32_t s0, s1;
+      scatter_selectors(static_cast<uint32_t>(i), K, s0, s1);
+      sel_one[i] = make_uint2(s0, s1);
+    }
+    for (int i = tid; i < 2 * 16 * 16; i += 288) (&s_acc[0][0][0])[i] = 0;
+    asm volatile("bar.sync 1, 288;" ::: "memory");
+    uint2* tab = reinterpret_cast<uint2*>(sel_bytes);
+    for (int i = tid; i < kSelEntries * 32; i += 288) tab[i] = sel_one[i >> 5];
+    asm volatile("bar.sync 1, 288;" ::: "memory");
+  }
+  const int total = grp.unit_start[grp.count];
   auto problem_of = [&](int unit) {
     int pi = 0;
-    while (pi + 1 < grp.count && unit >= grp.block_start[pi + 1]) ++pi;
+    while (pi + 1 < grp.count && unit >= grp.unit_start[pi + 1]) ++pi;
     return pi;
   };
 
   if (warp == 8) {
-    // ---------------- producer
+    // ---------------- producer (packed weights only: safe before griddepcontrol.wait)
     if (lane == 0) {
       int it = 0;
       bool ok = true;
       for (int unit = blockIdx.x; unit < total && ok; unit += gridDim.x) {
         const int pi = problem_of(unit);
-        const int row0 = (unit - grp.block_start[pi]) * 16;
+        const int rows = grp.p[pi].rows;
+        const int row0 = (unit - grp.unit_start[pi]) * rows;
         const int nkt = (grp.p[pi].d_in / 8 + kTileChunks - 1) / kTileChunks;
         for (int kt = 0; kt < nkt; ++kt, ++it) {
-          const int s = it % kGemvStages;
-          if (!mbar_wait(&s_empty[s], (static_cast<uint32_t>(it / kGemvStages) & 1u) ^ 1u, &s_abort, err)) {
+          const int s = it % Tl::STAGES;
+          if (!mbar_wait_sleep(&s_empty[s], (static_cast<uint32_t>(it / Tl::STAGES) & 1u) ^ 1u, &s_abort, err)) {
             ok = false;
             break;
           }
           uint8_t* st = ring + s * Tl::BYTES;
-          mbar_arrive_expect_tx(&s_full[s], Tl::BYTES);
+          mbar_arrive_expect_tx(&s_full[s], rows * (Tl::CODE_ROW + Tl::INDEX_ROW));
           tma_load_2d(st, &grp.tm_codes[pi], &s_full[s], kt * (Tl::CODE_ROW / 4), row0);
           tma_load_2d(st + 16 * Tl::CODE_ROW, &grp.tm_index[pi], &s_full[s], kt * (Tl::INDEX_ROW / 4), row0);
         }
       }
       if (!ok) {
-        for (int i = (it > kGemvStages ? it - kGemvStages : 0); i < it; ++i)
-          mbar_wait(&s_full[i % kGemvStages], static_cast<uint32_t>(i / kGemvStages) & 1u, nullptr, err);
+        for (int i = (it > Tl::STAGES ? it - Tl::STAGES : 0); i < it; ++i)
+          mbar_wait(&s_full[i % Tl::STAGES], static_cast<uint32_t>(i / Tl::STAGES) & 1u, nullptr, err);
       }
     }
-    return;  // the producer warp takes no part in the consumers' named barrier
+    return;
+  }
+
+  griddep_wait();  // activations, scales and outputs may come from / go to the previous kernel
+
+  if (warp == 9) {
+    // ---------------- epilogue: scale and store the sums of every unit
+    for (int i = lane; i < grp.count * 16; i += 32) {
+      const int pi = i >> 4, tok = i & 15;
+      s_scale[pi][tok] =
+          tok < grp.batch ? __fmul_rn(*grp.p[pi].gamma, __fdiv_rn(grp.p[pi].amax[tok], 127.0f)) : 0.0f;
+    }
+    __syncwarp();
+    int u = 0;
+    for (int unit = blockIdx.x; unit < total; unit += gridDim.x, ++u) {
+      const int b = u & 1;
+      if (!mbar_wait_sleep(&s_accf[b], static_cast<uint32_t>(u >> 1) & 1u, &s_abort, err)) break;
+      const int pi = problem_of(unit);
+      const GemvProblemDev& P = grp.p[pi];
+      const int rows = P.rows;
+      const int row0 = (unit - grp.unit_start[pi]) * rows;
+      for (int i = lane; i < rows * grp.batch; i += 32) {
+        const int r = i / grp.batch, tok = i - r * grp.batch;
+        const int v = s_acc[b][r][tok];
+        s_acc[b][r][tok] = 0;
+        if (row0 + r < P.d_out)
+          P.Y[static_cast<size_t>(tok) * P.d_out + row0 + r] = __fmul_rn(__int2float_rn(v), s_scale[pi][tok]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_acce[b]);
+    }
+    return;
   }
 
   // ---------------- consumers (warps 0-7)
   const int g = lane >> 2, t = lane & 3;
-  int it = 0;
-  for (int unit = blockIdx.x; unit < total; unit += gridDim.x) {
+  const uint32_t lane8 = static_cast<uint32_t>(lane) * 8u;
+  int it = 0, u = 0;
+  for (int unit = blockIdx.x; unit < total; unit += gridDim.x, ++u) {
     const int pi = problem_of(unit);
     const GemvProblemDev& P = grp.p[pi];
-    const int row0 = (unit - grp.block_start[pi]) * 16;
-    const int d_in = P.d_in, d_out = P.d_out;
+    const bool two = P.rows == 16;  // rows g and g + 8, else rows g only
+    const int d_in = P.d_in;
     const int nchunks = d_in / 8;
     const int nkt = (nchunks + kTileChunks - 1) / kTileChunks;
 
@@ -282,124 +393,65 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
 #pragma unroll
       for (int n = 0; n < NT; ++n) acc[e][n][0] = acc[e][n][1] = acc[e][n][2] = acc[e][n][3] = 0;
 
-    const uint2* xr[NT];
+    const uint8_t* xr[NT];
     bool tv[NT];
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       const int tok = n * 8 + g;
       tv[n] = tok < grp.batch;
-      xr[n] = reinterpret_cast<const uint2*>(P.Xq + static_cast<size_t>(tv[n] ? tok : 0) * d_in);
+      xr[n] = reinterpret_cast<const uint8_t*>(P.Xq) + static_cast<size_t>(tv[n] ? tok : 0) * d_in;
     }
     bool ok = true;
     for (int kt = 0; kt < nkt; ++kt, ++it) {
-      const int s = it % kGemvStages;
-      if (!mbar_wait(&s_full[s], static_cast<uint32_t>(it / kGemvStages) & 1u, &s_abort, err)) {
+      const int s = it % Tl::STAGES;
+      // activations of this lane's 8 chunks (64 bytes per token), issued before the wait
+      const int chl = kt * kTileChunks + warp * 32 + 8 * t;
+      uint4 xv[NT][4];
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          xv[n][q] = make_uint4(0u, 0u, 0u, 0u);
+          if (tv[n] && chl + 2 * q < nchunks)
+            xv[n][q] = __ldg(reinterpret_cast<const uint4*>(xr[n] + static_cast<size_t>(chl + 2 * q) * 8));
+        }
+      if (!mbar_wait_sleep(&s_full[s], static_cast<uint32_t>(it / Tl::STAGES) & 1u, &s_abort, err)) {
         ok = false;
         break;
       }
       const uint8_t* st = ring + s * Tl::BYTES;
-      const int ch0 = kt * kTileChunks + warp * 32 + 8 * t;  // this lane's first chunk (global index)
-      // code words and index bytes of rows g and g + 8 for chunks ch0 .. ch0 + 7
-      const int coff = (warp * 32 + 8 * t) * 2 * K / 8;
-      uint32_t wa[5] = {0u, 0u, 0u, 0u, 0u}, wb[5] = {0u, 0u, 0u, 0u, 0u};
-      if constexpr ((K & 1) == 0) {
-#pragma unroll
-        for (int i = 0; i < K / 2; ++i) {
-          wa[i] = *reinterpret_cast<const uint32_t*>(st + g * Tl::CODE_ROW + coff + 4 * i);
-          wb[i] = *reinterpret_cast<const uint32_t*>(st + (g + 8) * Tl::CODE_ROW + coff + 4 * i);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < K; ++i) {
-          wa[i >> 1] |= static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(st + g * Tl::CODE_ROW + coff + 2 * i))
-                        << (16 * (i & 1));
-          wb[i >> 1] |= static_cast<uint32_t>(
-                             *reinterpret_cast<const uint16_t*>(st + (g + 8) * Tl::CODE_ROW + coff + 2 * i))
-                         << (16 * (i & 1));
-        }
-      }
-      const uint8_t* ib = st + 16 * Tl::CODE_ROW;
-      const uint2 ma = *reinterpret_cast<const uint2*>(ib + g * Tl::INDEX_ROW + warp * 32 + 8 * t);
-      const uint2 mb = *reinterpret_cast<const uint2*>(ib + (g + 8) * Tl::INDEX_ROW + warp * 32 + 8 * t);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t ca = chunk_codes<K>(wa, j), cb = chunk_codes<K>(wb, j);
-        const uint32_t mA = ((j < 4 ? ma.x : ma.y) >> (8 * (j & 3))) & 0xFFu;
-        const uint32_t mB = ((j < 4 ? mb.x : mb.y) >> (8 * (j & 3))) & 0xFFu;
-        // slot values v0..v(K-1) as bytes of (lo, hi); byte 7 stays 0 (K <= 7)
-        uint32_t alo, ahi, blo, bhi;
-        {
-          const uint32_t a0 = s_code[((ca & 63u) << 5) + lane];
-          const uint32_t b0v = s_code[((cb & 63u) << 5) + lane];
-          if constexpr (K <= 3) {
-            alo = a0; ahi = 0u; blo = b0v; bhi = 0u;
-          } else {
-            const uint32_t a1 = s_code[(((ca >> 6) & 63u) << 5) + lane];
-            const uint32_t b1v = s_code[(((cb >> 6) & 63u) << 5) + lane];
-            alo = a0 | (a1 << 24);
-            blo = b0v | (b1v << 24);
-            ahi = a1 >> 8;
-            bhi = b1v >> 8;
-            if constexpr (K > 6) {
-              const uint32_t a2 = s_code[(((ca >> 12) & 63u) << 5) + lane];
-              const uint32_t b2 = s_code[(((cb >> 12) & 63u) << 5) + lane];
-              ahi |= a2 << 16;
-              bhi |= b2 << 16;
-            }
-          }
-        }
-        const uint32_t selA = s_sel[(mA << 5) + lane], selB = s_sel[(mB << 5) + lane];
-        const uint32_t a_lo = __byte_perm(alo, ahi, selA & 0xFFFFu), a_hi = __byte_perm(alo, ahi, selA >> 16);
-        const uint32_t b_lo = __byte_perm(blo, bhi, selB & 0xFFFFu), b_hi = __byte_perm(blo, bhi, selB >> 16);
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          const uint2 x = (tv[n] && ch0 + j < nchunks) ? __ldg(xr[n] + ch0 + j) : make_uint2(0u, 0u);
-          mma_s8_16x8x32(acc[j & 1][n], a_lo, b_lo, a_hi, b_hi, x.x, x.y);
-        }
-      }
+      if (two)
+        gemv_tile<K, NT, true>(acc, st, sel_bytes, xv, warp, g, t, lane8);
+      else
+        gemv_tile<K, NT, false>(acc, st, sel_bytes, xv, warp, g, t, lane8);
       // Free the stage only now: every value read from it has been used by the
       // decode above, so no load of this warp can still be pending when the
       // next TMA copy overwrites the stage.
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[s]);
     }
+    if (!ok) break;
+    // hand the unit's partial sums to the epilogue warp
+    const int b = u & 1;
+    if (!mbar_wait_sleep(&s_acce[b], (static_cast<uint32_t>(u >> 1) & 1u) ^ 1u, &s_abort, err)) break;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-      s_part[warp][g][n * 8 + 2 * t] = acc[0][n][0] + acc[1][n][0];
-      s_part[warp][g][n * 8 + 2 * t + 1] = acc[0][n][1] + acc[1][n][1];
-      s_part[warp][g + 8][n * 8 + 2 * t] = acc[0][n][2] + acc[1][n][2];
-      s_part[warp][g + 8][n * 8 + 2 * t + 1] = acc[0][n][3] + acc[1][n][3];
-    }
-    // Barrier of the 8 consumer warps that also agrees on giving up: every
-    // consumer reaches it, so a timed-out wait in one warp cannot strand the
-    // others at a barrier.
-    uint32_t any_fail;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 256, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(any_fail)
-        : "r"(ok ? 0u : 1u)
-        : "memory");
-    if (any_fail) break;
-    if (threadIdx.x < 16 * grp.batch) {
-      const int r = threadIdx.x / grp.batch, tok = threadIdx.x - r * grp.batch;
-      const int row = row0 + r;
-      if (row < d_out) {
-        int sum = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) sum += s_part[w][r][tok];
-        const float sc = __fmul_rn(*P.gamma, __fdiv_rn(P.amax[tok], 127.0f));
-        P.Y[static_cast<size_t>(tok) * d_out + row] = __fmul_rn(__int2float_rn(sum), sc);
+      atomicAdd(&s_acc[b][g][n * 8 + 2 * t], acc[0][n][0] + acc[1][n][0]);
+      atomicAdd(&s_acc[b][g][n * 8 + 2 * t + 1], acc[0][n][1] + acc[1][n][1]);
+      if (two) {
+        atomicAdd(&s_acc[b][g + 8][n * 8 + 2 * t], acc[0][n][2] + acc[1][n][2]);
+        atomicAdd(&s_acc[b][g + 8][n * 8 + 2 * t + 1], acc[0][n][3] + acc[1][n][3]);
       }
     }
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s_accf[b]);
   }
 }
 
 template <int K>
 cudaError_t launch_gemv_k(const GemvGroup& grp, int units, int num_sms, cudaStream_t stream, uint32_t* err) {
   auto kern = grp.batch <= 8 ? gemv_packed_kernel<K, 1> : gemv_packed_kernel<K, 2>;
-  const int smem = kGemvStages * GemvTile<K>::BYTES + (kCodeEntries + kSelEntries) * 32 * 4 + 128;
+  const int smem = GemvTile<K>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -408,8 +460,19 @@ cudaError_t launch_gemv_k(const GemvGroup& grp, int units, int num_sms, cudaStre
   if (per_sm < 1) per_sm = 1;
   int blocks = num_sms * per_sm;  // persistent
   if (blocks > units) blocks = units;
-  kern<<<blocks, kGemvThreads, smem, stream>>>(grp, err);
-  return cudaGetLastError();
+  // Programmatic dependent launch: this grid may start while the previous
+  // kernel of the stream finishes (see the kernel's griddepcontrol.wait).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, grp, err);
 }
 
 }  // namespace
@@ -439,20 +502,39 @@ cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch,
     GemvGroup grp{};
     grp.count = (count - c0) < kGemvMaxGroup ? (count - c0) : kGemvMaxGroup;
     grp.batch = batch;
+    // Unit rows: 8 for problems whose K is at least twice the shortest K of
+    // the launch, else 16; units are numbered heaviest (rows x K) first.
+    int min_chunks = 1 << 30;
+    for (int i = 0; i < grp.count; ++i) min_chunks = min(min_chunks, probs[c0 + i].d_in / 8);
+    int order[kGemvMaxGroup];
+    long long work[kGemvMaxGroup];
+    for (int i = 0; i < grp.count; ++i) {
+      const int nch = probs[c0 + i].d_in / 8;
+      const int rows = nch >= 2 * min_chunks ? 8 : 16;
+      work[i] = static_cast<long long>(rows) * nch;
+      order[i] = i;
+    }
+    for (int i = 1; i < grp.count; ++i)  // insertion sort, heaviest first, stable
+      for (int j = i; j > 0 && work[order[j]] > work[order[j - 1]]; --j) {
+        const int tmp = order[j];
+        order[j] = order[j - 1];
+        order[j - 1] = tmp;
+      }
     int units = 0;
     for (int i = 0; i < grp.count; ++i) {
-      GemvProblemDev p = probs[c0 + i];
+      GemvProblemDev p = probs[c0 + order[i]];
       p.crow = packed_codes_row_bytes(p.d_in, N, M);
       p.irow = packed_index_row_bytes(p.d_in, M);
+      p.rows = p.d_in / 8 >= 2 * min_chunks ? 8 : 16;
       grp.p[i] = p;
-      grp.block_start[i] = units;
-      units += (p.d_out + 15) / 16;
-      if (!make_tmap_u32(&grp.tm_codes[i], p.packed, p.crow / 4, p.d_out, p.crow, code_tile_words, 16) ||
+      grp.unit_start[i] = units;
+      units += (p.d_out + p.rows - 1) / p.rows;
+      if (!make_tmap_u32(&grp.tm_codes[i], p.packed, p.crow / 4, p.d_out, p.crow, code_tile_words, p.rows) ||
           !make_tmap_u32(&grp.tm_index[i], p.packed + static_cast<size_t>(p.d_out) * p.crow, p.irow / 4, p.d_out,
-                         p.irow, index_tile_words, 16))
+                         p.irow, index_tile_words, p.rows))
         return cudaErrorInvalidValue;
     }
-    grp.block_start[grp.count] = units;
+    grp.unit_start[grp.count] = units;
     if (units == 0) continue;
     cudaError_t e;
     switch (K) {

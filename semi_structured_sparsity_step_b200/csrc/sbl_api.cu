@@ -306,7 +306,7 @@ sbl_status sbl_gemv_packed_group(const sbl_gemv_problem* problems, int count, in
     if (!aligned16(p.Xq) || !aligned16(p.amax) || !aligned16(p.packed) || !aligned16(p.Y) ||
         (reinterpret_cast<uintptr_t>(p.gamma) & 3u) != 0)
       return SBL_ERR_ALIGN;
-    dev[i] = GemvProblemDev{p.packed, p.Xq, p.amax, p.gamma, p.Y, p.d_in, p.d_out, 0, 0};
+    dev[i] = GemvProblemDev{p.packed, p.Xq, p.amax, p.gamma, p.Y, p.d_in, p.d_out, 0, 0, 0};
   }
   DeviceInfo* d = nullptr;
   if ((st = current_device(&d)) != SBL_OK) return st;

@@ -84,6 +84,43 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait for waits that are expected to be long (a consumer waiting for
+// HBM, a producer waiting for a free stage): try_wait with a suspend-time
+// hint, so the waiting warp sleeps in the barrier unit instead of spinning
+// and taking issue slots from the warps that do work.  The hint (20 us) is
+// an upper bound per try; the time limit is checked after every try.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                uint32_t* err) {
+  if (mbar_try_wait_sleep(bar, parity)) return true;
+  uint64_t t0 = 0;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((it & 63u) == 0) {  // the abort flag and the clock are read every 64 tries only
+      if (abort != nullptr && *abort) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        latch_error(err, kErrTimeout);
+        if (abort != nullptr) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // ----------------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion on an mbarrier.
 // c0 is the innermost (contiguous) coordinate in elements; c0 * element size

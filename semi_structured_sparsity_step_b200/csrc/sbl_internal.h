@@ -71,6 +71,7 @@ struct GemvProblemDev {
   float* Y;
   int d_in, d_out;
   size_t crow, irow;  // filled in by the launcher
+  int rows;           // rows per work unit (16 or 8), filled in by the launcher
 };
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
                               cudaStream_t stream, int num_sms, uint32_t* err);

@@ -251,12 +251,13 @@ def test_gamma_exact_on_log_uniform_magnitudes(lib):
         assert np.array_equal(L.W_eff.cpu().numpy(), weff)
 
 
-def test_gemv_group_matches_single_calls(lib):
+@pytest.mark.parametrize("batch", [5, 16])
+def test_gemv_group_matches_single_calls(lib, batch):
     """One grouped launch over projections of different shapes equals the
-    per-projection results (and the oracle)."""
+    oracle.  The long-K problems run as 8-row units, the shortest as 16-row
+    units, so both unit shapes are covered, with one and two token tiles."""
     shapes = [(264, 2048), (8, 896), (520, 11008), (136, 4864)]
     probs, refs = [], []
-    batch = 5
     for i, (d_out, d_in) in enumerate(shapes):
         w = synth.trimodal_weight(d_out, d_in, seed=30, tensor_id=i)
         weff, gamma, _ = oracle.effective_weight(synth.bits(w), 6, 8)
