@@ -5,9 +5,12 @@ One step = the whole hot path over one batch of the Qwen2.5-3B-shaped layer
 set (q/o 2048x2048, k/v 256x2048, gate/up 11008x2048, down 2048x11008),
 32768 tokens (16 x 2048), 6:8:
 
-  for every projection:  sbl_mask_quant   (mask, gamma, ternary, quant-then-mask)
-  for every input:       sbl_act_quant    (attn_in, o_in, mlp_in, down_in)
-  for every projection:  sbl_forward      (int8 tcgen05 product)
+  for every projection:  sbl_mask_quant   (mask, gamma, ternary, quant-then-mask;
+                                           on three side streams)
+  for every input:       sbl_act_quant    (attn_in, o_in, mlp_in, down_in; main
+                                           stream, overlapped with the above)
+  for every projection:  sbl_forward      (int8 tcgen05 product; at N:M = 2:4,
+                                           sbl_compress24 + the sparse MMA)
                          sbl_backward     (bf16 tcgen05 dX, then dW)
 
 Inputs are seeded synthetic tensors (synth): trimodal bf16 master weights,
@@ -107,6 +110,11 @@ class Step:
         self.dX = {p.name: torch.empty(T, p.d_in, dtype=torch.float32, device=dev) for p in ls.projections}
         self.dW = {p.name: torch.empty(p.d_out, p.d_in, dtype=torch.float32, device=dev) for p in ls.projections}
         n_p, n_x = len(ls.projections), len(ls.inputs)
+        # the weight steps (mask, gamma, ternary) of the projections are
+        # independent of the activation quantisation: they run on side streams,
+        # overlapped with act_quant on the main stream, and join before the
+        # forward products
+        self.side = [torch.cuda.Stream() for _ in range(3)]
         self.sparse24 = (N_KEEP, M_GROUP) == (2, 4)  # compress + sparse tensor-core forward
         self.kernels_per_step = 2 * n_p + n_x + 3 * n_p + (n_p if self.sparse24 else 0)
 
@@ -125,11 +133,21 @@ class Step:
             b.record(stream)
             ev.setdefault(name, []).append((a, b))
 
-        for p in ls.projections:
-            timed("mask_quant", lambda p=p: self.layers[p.name].weight_step(stream))
-        for n, d in ls.inputs.items():
-            timed("act_quant", lambda n=n, d=d: sbl.sbl_act_quant(self.X[n], T, d, self.Xq[n], self.amax[n],
-                                                                  stream))
+        def weight_and_act_quant():
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            for sd in self.side:
+                sd.wait_event(fork)
+            for i, p in enumerate(ls.projections):
+                self.layers[p.name].weight_step(self.side[i % len(self.side)])
+            for n, d in ls.inputs.items():
+                sbl.sbl_act_quant(self.X[n], T, d, self.Xq[n], self.amax[n], stream)
+            for sd in self.side:
+                join = torch.cuda.Event()
+                join.record(sd)
+                stream.wait_event(join)
+
+        timed("weight_and_act_quant", weight_and_act_quant)
         for p in ls.projections:
             L = self.layers[p.name]
             timed("forward_i8", lambda p=p, L=L: L.forward(self.Xq[p.input_name], self.amax[p.input_name],
@@ -369,10 +387,12 @@ def run_decode(args):
 def run_prefill(args):
     """Prefill forward on the packed 6:8 format of the 3B layer set: per
     projection, int8 activations (absmax-quantised N(0, 1)) times the packed
-    weight expanded in shared memory (sbl_forward_packed), against the same
-    product from the unpacked int8 W_eff (sbl_forward).  Shapes: 512 tokens
-    (1 x 512), 8192 (8 x 1024) and 32768 (16 x 2048).  One pass = the seven
-    projections; int8 ops = 2 T P (dense-equivalent)."""
+    weight, three ways: expanded in shared memory for every token tile
+    (sbl_forward_packed), unpacked once per pass and multiplied by the dense
+    int8 kernel (sbl_unpack + sbl_forward), and from an int8 W_eff that is
+    already resident (sbl_forward).  Shapes: 512 tokens (1 x 512), 8192
+    (8 x 1024) and 32768 (16 x 2048).  One pass = the seven projections,
+    captured in a CUDA graph; int8 ops = 2 T P (dense-equivalent)."""
     import semi_structured_sparsity_step_b200 as sbl
     from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer, act_quant
     torch.cuda.set_device(0)
@@ -388,6 +408,7 @@ def run_prefill(args):
         pk = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
         sbl.sbl_pack(L.W_eff, p.d_out, p.d_in, N_KEEP, M_GROUP, pk, nbytes)
         layers.append((p, L, pk))
+    unpacked = [torch.empty(p.d_out, p.d_in, dtype=torch.int8, device="cuda") for (p, _, _) in layers]
     sbl.sbl_check()
     pk_peak = peaks()
     i8_peak = pk_peak["bf16"] * NOMINAL_I8_OVER_BF16  # burst: each pass is timed on its own
@@ -403,19 +424,28 @@ def run_prefill(args):
             xs[n] = (xq, am)
         ys = [torch.empty(T, p.d_out, dtype=torch.float32, device="cuda") for (p, _, _) in layers]
 
-        def one_pass(packed):
-            for (p, L, pk), y in zip(layers, ys):
+        def one_pass(variant):
+            for (p, L, pk), y, wk in zip(layers, ys, unpacked):
                 xq, am = xs[p.input_name]
-                if packed:
+                if variant == "packed":      # weight decoded in shared memory for every token tile
                     sbl.sbl_forward_packed(xq, am, pk, L.gamma, T, p.d_in, p.d_out, N_KEEP, M_GROUP, y, None, stream)
-                else:
+                elif variant == "unpack_int8":  # decoded once per pass, then the dense int8 product
+                    sbl.sbl_unpack(pk, p.d_out, p.d_in, N_KEEP, M_GROUP, wk, stream)
+                    sbl.sbl_forward(xq, am, wk, L.gamma, T, p.d_in, p.d_out, y, None, stream)
+                else:                        # int8 W_eff already resident (training layout)
                     sbl.sbl_forward(xq, am, L.W_eff, L.gamma, T, p.d_in, p.d_out, y, None, stream)
 
         row = {}
-        for packed in (True, False):
+        for variant in ("packed", "unpack_int8", "int8_weff"):
             with torch.cuda.stream(stream):
-                for _ in range(args.warmup):
-                    one_pass(packed)
+                for _ in range(2):
+                    one_pass(variant)
+            stream.synchronize()
+            graph = torch.cuda.CUDAGraph()  # one pass per replay: no host launch cost in the timing
+            with torch.cuda.graph(graph, stream=stream):
+                one_pass(variant)
+            for _ in range(args.warmup):
+                graph.replay()
             stream.synchronize()
             reps = max(args.steps, 5)
             e0 = torch.cuda.Event(enable_timing=True)
@@ -423,13 +453,14 @@ def run_prefill(args):
             e0.record(stream)
             with torch.cuda.stream(stream):
                 for _ in range(reps):
-                    one_pass(packed)
+                    graph.replay()
             e1.record(stream)
             stream.synchronize()
+            del graph
             ms = e0.elapsed_time(e1) / reps
             tops = 2.0 * T * ls.params / (ms / 1e3) / 1e12
-            row["packed" if packed else "int8_weff"] = {"ms_per_pass": ms, "tokens_per_s": T / (ms / 1e3),
-                                                         "int8_tops": tops, "frac_int8_peak": tops / i8_peak}
+            row[variant] = {"ms_per_pass": ms, "tokens_per_s": T / (ms / 1e3), "int8_tops": tops,
+                            "frac_int8_peak": tops / i8_peak}
         sbl.sbl_check()
         results[str(T)] = row
         del xs, ys

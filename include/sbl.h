@@ -247,8 +247,24 @@ size_t sbl_packed_bytes(int d_out, int d_in, int N, int M);
 sbl_status sbl_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M,
                     uint8_t* packed, size_t packed_bytes, void* stream);
 
+/* Unpack: the packed format back to int8 W_eff [d_out, d_in] (bit for bit
+ * the W_eff that was packed).  [article] 7.1 (the cached format is decoded
+ * where it is used).  For prefill over many tokens, unpacking once and
+ * calling sbl_forward is faster than sbl_forward_packed, which decodes the
+ * weight again for every 256-token tile.
+ *   packed  sbl_pack output of the [d_out, d_in] weight, N:M as packed.
+ *   W_eff   [d_out, d_in] int8 out. */
+sbl_status sbl_unpack(const uint8_t* packed, int d_out, int d_in, int N, int M,
+                      int8_t* W_eff, void* stream);
+
 /* Decode GEMV on the packed format, batch 1..16 tokens.
  * [summary] 实验结果 / Table 3 (decode on the 6:8 ternary model).
+ * The kernel is launched with programmatic dependent launch: it may start
+ * while the previous kernel of `stream` is finishing, build its tables and
+ * begin streaming `packed`; it reads Xq, amax and gamma and writes Y only
+ * after that kernel has completed.  No kernel of this library that lets its
+ * successor start early writes a packed buffer, so plain stream order is
+ * enough for every sequence of library calls.
  *   Xq [batch, d_in] int8, amax [batch] float, gamma 1 float (device),
  *   Y  [batch, d_out] float out, same formula as sbl_forward. */
 sbl_status sbl_gemv_packed(const int8_t* Xq, const float* amax, int batch,

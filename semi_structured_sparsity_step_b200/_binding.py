@@ -44,6 +44,7 @@ SIGNATURES = {
     "sbl_backward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp, _c_size, _vp]),
     "sbl_packed_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "sbl_pack": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
+    "sbl_unpack": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "sbl_gemv_packed": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "sbl_gemv_packed_group": (_c_int, [ctypes.POINTER(GemvProblem), _c_int, _c_int, _c_int, _c_int, _vp]),
 }
@@ -185,6 +186,10 @@ def sbl_packed_bytes(d_out, d_in, N, M) -> int:
 
 def sbl_pack(W_eff, d_out, d_in, N, M, packed, packed_bytes, stream=None) -> None:
     _call("sbl_pack", _ptr(W_eff), d_out, d_in, N, M, _ptr(packed), packed_bytes, _stream(stream))
+
+
+def sbl_unpack(packed, d_out, d_in, N, M, W_eff, stream=None) -> None:
+    _call("sbl_unpack", _ptr(packed), d_out, d_in, N, M, _ptr(W_eff), _stream(stream))
 
 
 def sbl_gemv_packed(Xq, amax, batch, packed, gamma, d_in, d_out, N, M, Y, stream=None) -> None:

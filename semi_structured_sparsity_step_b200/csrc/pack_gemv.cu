@@ -475,6 +475,65 @@ cudaError_t launch_gemv_k(const GemvGroup& grp, int units, int num_sms, cudaStre
   return cudaLaunchKernelEx(&cfg, kern, grp, err);
 }
 
+// ----------------------------------------------------------------- unpack
+// Packed format -> int8 W_eff [d_out, d_in] (the operand of the dense int8
+// forward), for prefill: decoding a weight once and running the dense
+// tensor-core product is cheaper than decoding it again for every token
+// tile.  One thread per run of 8 chunks (64 weights) of a row: its 2K code
+// bytes and 8 mask bytes are read with plain loads, each chunk is decoded by
+// packed_decode.cuh (selector table in shared memory, one copy), and the 64
+// bytes are stored with four 16-byte stores.  HBM bound.
+template <int K>
+__global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__ packed, int d_out, int d_in,
+                                                     size_t crow, size_t irow, int8_t* __restrict__ W) {
+  __shared__ uint2 s_sel[256];
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+    uint32_t s0, s1;
+    scatter_selectors(static_cast<uint32_t>(i), K, s0, s1);
+    s_sel[i] = make_uint2(s0, s1);
+  }
+  __syncthreads();
+  const int nch = d_in / 8;
+  const int runs_per_row = (nch + 7) / 8;
+  const long long total = static_cast<long long>(d_out) * runs_per_row;
+  const uint8_t* index = packed + static_cast<size_t>(d_out) * crow;
+  for (long long it = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; it < total;
+       it += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(it / runs_per_row);
+    const int c0 = static_cast<int>(it - static_cast<long long>(row) * runs_per_row) * 8;
+    const int nc = min(8, nch - c0);
+    // code bits of chunks c0 .. c0 + nc - 1 (2K bits each, starting at a byte boundary: c0 % 8 == 0)
+    uint32_t w[5] = {0u, 0u, 0u, 0u, 0u};
+    uint8_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const uint8_t* cr = packed + static_cast<size_t>(row) * crow + static_cast<size_t>(c0) * 2 * K / 8;
+    const uint8_t* mr = index + static_cast<size_t>(row) * irow + c0;
+    if ((K & 1) == 0 && nc == 8) {
+      // a full run: 2K code bytes at a 4-byte aligned offset, 8 mask bytes at an 8-byte aligned one
+#pragma unroll
+      for (int i = 0; i < K / 2; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t*>(cr) + i);
+      const uint2 mm = __ldg(reinterpret_cast<const uint2*>(mr));
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m[j] = static_cast<uint8_t>(((j < 4 ? mm.x : mm.y) >> (8 * (j & 3))) & 0xFFu);
+    } else {
+      const int cbytes = (nc * 2 * K + 7) / 8;
+      for (int b = 0; b < cbytes; ++b) w[b >> 2] |= static_cast<uint32_t>(cr[b]) << (8 * (b & 3));
+      for (int j = 0; j < nc; ++j) m[j] = mr[j];
+    }
+    int8_t* out = W + static_cast<size_t>(row) * d_in + static_cast<size_t>(c0) * 8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= nc) break;
+      const int bit = 2 * K * j;
+      const int wi = bit >> 5, sh = bit & 31;
+      const uint32_t v = sh == 0 ? w[wi] : __funnelshift_r(w[wi], w[wi + 1], sh);
+      uint32_t lo, hi;
+      ChunkCodes<K>::decode(v, lo, hi);
+      const uint2 sel = s_sel[m[j]];
+      *reinterpret_cast<uint2*>(out + 8 * j) = make_uint2(prmt(lo, hi, sel.x), prmt(lo, hi, sel.y));
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M, uint8_t* packed,
@@ -550,6 +609,29 @@ cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch,
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_unpack(const uint8_t* packed, int d_out, int d_in, int N, int M, int8_t* W_eff,
+                          cudaStream_t stream, int num_sms) {
+  if (d_out == 0 || d_in == 0) return cudaSuccess;
+  const size_t crow = packed_codes_row_bytes(d_in, N, M);
+  const size_t irow = packed_index_row_bytes(d_in, M);
+  const long long runs = static_cast<long long>(d_out) * ((d_in / 8 + 7) / 8);
+  long long blocks = (runs + 255) / 256;
+  const long long cap = static_cast<long long>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  const unsigned nb = static_cast<unsigned>(blocks);
+  switch (8 * N / M) {
+    case 1: unpack_kernel<1><<<nb, 256, 0, stream>>>(packed, d_out, d_in, crow, irow, W_eff); break;
+    case 2: unpack_kernel<2><<<nb, 256, 0, stream>>>(packed, d_out, d_in, crow, irow, W_eff); break;
+    case 3: unpack_kernel<3><<<nb, 256, 0, stream>>>(packed, d_out, d_in, crow, irow, W_eff); break;
+    case 4: unpack_kernel<4><<<nb, 256, 0, stream>>>(packed, d_out, d_in, crow, irow, W_eff); break;
+    case 5: unpack_kernel<5><<<nb, 256, 0, stream>>>(packed, d_out, d_in, crow, irow, W_eff); break;
+    case 6: unpack_kernel<6><<<nb, 256, 0, stream>>>(packed, d_out, d_in, crow, irow, W_eff); break;
+    case 7: unpack_kernel<7><<<nb, 256, 0, stream>>>(packed, d_out, d_in, crow, irow, W_eff); break;
+    default: unpack_kernel<8><<<nb, 256, 0, stream>>>(packed, d_out, d_in, crow, irow, W_eff); break;
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gemv_packed(const int8_t* Xq, const float* amax, int batch, const uint8_t* packed,

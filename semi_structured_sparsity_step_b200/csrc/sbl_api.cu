@@ -271,6 +271,19 @@ sbl_status sbl_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M, uint
   return from_cuda(launch_pack(W_eff, d_out, d_in, N, M, packed, static_cast<cudaStream_t>(stream), d->err));
 }
 
+sbl_status sbl_unpack(const uint8_t* packed, int d_out, int d_in, int N, int M, int8_t* W_eff, void* stream) {
+  sbl_status st = check_nm(N, M);
+  if (st != SBL_OK) return st;
+  if ((st = check_dims(d_in, d_out)) != SBL_OK) return st;
+  if (d_in % M != 0) return SBL_ERR_SHAPE;
+  if (d_out == 0 || d_in == 0) return SBL_OK;
+  if (packed == nullptr || W_eff == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(W_eff)) return SBL_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  return from_cuda(launch_unpack(packed, d_out, d_in, N, M, W_eff, static_cast<cudaStream_t>(stream), d->num_sms));
+}
+
 sbl_status sbl_gemv_packed(const int8_t* Xq, const float* amax, int batch, const uint8_t* packed,
                            const float* gamma, int d_in, int d_out, int N, int M, float* Y, void* stream) {
   sbl_status st = check_nm(N, M);

@@ -61,6 +61,8 @@ cudaError_t launch_forward_sparse24(const int8_t* Xq, const float* amax, const u
 // ---- packed format (pack_gemv.cu)
 size_t packed_codes_row_bytes(int d_in, int N, int M);
 size_t packed_index_row_bytes(int d_in, int M);
+cudaError_t launch_unpack(const uint8_t* packed, int d_out, int d_in, int N, int M, int8_t* W_eff,
+                          cudaStream_t stream, int num_sms);
 cudaError_t launch_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M, uint8_t* packed,
                         cudaStream_t stream, uint32_t* err);
 struct GemvProblemDev {

@@ -299,3 +299,22 @@ def test_forward_from_packed_matches_oracle(lib, T, d_out, d_in, N, M):
     racc = oracle.forward_acc(xq, weff)
     assert np.array_equal(acc.cpu().numpy(), racc)
     assert np.array_equal(Y.cpu().numpy(), oracle.forward_out(racc, gamma, amax))
+
+
+@pytest.mark.parametrize("d_out,d_in,N,M", [
+    (8, 16, 6, 8), (264, 2064, 6, 8), (136, 400, 2, 4), (520, 1040, 8, 8), (72, 4864, 4, 8), (40, 272, 3, 8),
+    (16, 112, 1, 4), (24, 208, 3, 4),
+])
+def test_unpack_restores_weff(lib, d_out, d_in, N, M):
+    """sbl_unpack of sbl_pack gives back W_eff bit for bit (and the oracle's
+    unpack of the same bytes), including runs cut short by d_in % 64."""
+    w = synth.trimodal_weight(d_out, d_in, seed=70, tensor_id=d_in)
+    weff, _, _ = oracle.effective_weight(synth.bits(w), N, M)
+    nbytes = lib.sbl_packed_bytes(d_out, d_in, N, M)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    lib.sbl_pack(torch.from_numpy(weff).cuda(), d_out, d_in, N, M, packed, nbytes)
+    out = torch.full((d_out, d_in), 77, dtype=torch.int8, device="cuda")
+    lib.sbl_unpack(packed, d_out, d_in, N, M, out)
+    lib.sbl_check()
+    assert np.array_equal(out.cpu().numpy(), weff)
+    assert np.array_equal(oracle.unpack(packed.cpu().numpy(), d_out, d_in, N, M), weff)
