@@ -50,6 +50,7 @@ WORKLOADS = {
     "qwen2.5-3b-up": (8192, "trimodal", 0.001, 0.01),
 }
 N_KEEP, M_GROUP = 6, 8
+SPARSE24 = False  # --sparse24: 2:4 layers use the sparse tensor core
 METRIC = "Sparse-BitLinear fwd+bwd tokens/s (3B-shape, 6:8)"
 
 NOMINAL_I8_OVER_BF16 = 2.0  # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
@@ -103,7 +104,8 @@ class Step:
         self.sbl, self.ls, self.T = sbl, ls, T
         self.W, self.X, self.dY = W, X, dY
         dev = "cuda"
-        self.layers = {p.name: SparseBitLinearLayer(W[p.name], N_KEEP, M_GROUP) for p in ls.projections}
+        self.layers = {p.name: SparseBitLinearLayer(W[p.name], N_KEEP, M_GROUP, sparse24=SPARSE24)
+                       for p in ls.projections}
         self.Xq = {n: torch.empty(T, d, dtype=torch.int8, device=dev) for n, d in ls.inputs.items()}
         self.amax = {n: torch.empty(T, dtype=torch.float32, device=dev) for n in ls.inputs}
         self.Y = {p.name: torch.empty(T, p.d_out, dtype=torch.float32, device=dev) for p in ls.projections}
@@ -115,7 +117,7 @@ class Step:
         # overlapped with act_quant on the main stream, and join before the
         # forward products
         self.side = [torch.cuda.Stream() for _ in range(3)]
-        self.sparse24 = (N_KEEP, M_GROUP) == (2, 4)  # compress + sparse tensor-core forward
+        self.sparse24 = SPARSE24 and (N_KEEP, M_GROUP) == (2, 4)  # compress + sparse tensor-core forward
         self.kernels_per_step = 2 * n_p + n_x + 3 * n_p + (n_p if self.sparse24 else 0)
 
     def run(self, stream, ev=None):
@@ -509,9 +511,11 @@ def main():
     ap.add_argument("--mode", choices=["train", "decode", "prefill"], default="train")
     ap.add_argument("--layers", type=int, default=36, help="decode mode: distinct layer sets in the stack")
     ap.add_argument("--nm", default="6:8", help="N:M of the mask (the sweep: 8:8, 6:8, 4:8, 2:8, 2:4)")
+    ap.add_argument("--sparse24", action="store_true", help="2:4: forward on the sparse tensor core")
     args = ap.parse_args()
-    global N_KEEP, M_GROUP
+    global N_KEEP, M_GROUP, SPARSE24
     N_KEEP, M_GROUP = (int(v) for v in args.nm.split(":"))
+    SPARSE24 = args.sparse24
     if args.mode == "decode":
         run_decode(args)
         return
@@ -530,7 +534,8 @@ def main():
                           ", dY ~ N(0,1)",
               "tokens_per_step": T, "params": ls.params, "nm": f"{N_KEEP}:{M_GROUP}",
               "l2": "per-step working set larger than L2, no flush", "parallelism": f"dp{args.gpus} replicas",
-              "forward_kernel": ("2:4 compress + sparse int8 MMA (tcgen05.mma.sp)" if (N_KEEP, M_GROUP) == (2, 4)
+              "forward_kernel": ("2:4 compress + sparse int8 MMA (tcgen05.mma.sp)"
+                                 if SPARSE24 and (N_KEEP, M_GROUP) == (2, 4)
                                  else "dense int8 MMA (tcgen05.mma kind::i8)")}
 
     if args.impl == "reference":

@@ -207,6 +207,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSpThreads, 1)
     for (int w = pair_id; w < args.total; w += n_pairs, ++t) {
       const int mb = w % args.Mt, nb = w / args.Mt;
       const int b = t & 1;
+      // the tile's token scales, loaded while its MMAs still run: lane l holds
+      // the scale of token nb * kSpBN + 32 c + l in scl[c]
+      float scl[kSpBN / 32];
+#pragma unroll
+      for (int c = 0; c < kSpBN / 32; ++c) {
+        const int tl = nb * kSpBN + 32 * c + lane;
+        scl[c] = tl < args.T ? __ldg(args.amax + tl) : 0.0f;
+      }
+#pragma unroll
+      for (int c = 0; c < kSpBN / 32; ++c) scl[c] = __fmul_rn(g, __fdiv_rn(scl[c], 127.0f));
       if (!mbar_wait(&tfull[b], static_cast<uint32_t>(t >> 1) & 1u, abort_flag, args.err)) {
         give_up();
         break;
@@ -216,16 +226,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSpThreads, 1)
       const int o = mb * 256 + 128 * static_cast<int>(rank) + 32 * q + lane;
       const bool row_ok = o < args.d_out;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b * kSpBN);
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < kSpBN / 32; ++c) {
         const int t0 = nb * kSpBN + 32 * c;
         if (t0 >= args.T) break;  // warp-uniform
         uint32_t r[32];
         tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(32 * c), r);
         tmem_ld_wait();
-        // lane l holds the scale of token t0 + l
-        const int tl = t0 + lane;
-        const float sl = tl < args.T ? __fmul_rn(g, __fdiv_rn(args.amax[tl], 127.0f)) : 0.0f;
+        const float sl = scl[c];
         float* yc = args.Y + static_cast<long long>(t0) * args.d_out + o;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {

@@ -4,8 +4,8 @@ PyTorch only provides device memory and the stream here; every step of the
 operator runs in libsbl's kernels:
 
     weight_step()  -> sbl_mask_quant   (mask, gamma, ternary, quant-then-mask)
-                      + sbl_compress24 when N:M is 2:4
-    forward(X)     -> sbl_act_quant, sbl_forward (sbl_forward_sparse24 at 2:4)
+                      + sbl_compress24 for a 2:4 layer built with sparse24=True
+    forward(X)     -> sbl_act_quant, sbl_forward (or sbl_forward_sparse24)
     backward(dY)   -> sbl_backward     (dX and the dense dW)
 """
 from __future__ import annotations
@@ -16,7 +16,7 @@ from . import _binding as B
 
 
 class SparseBitLinearLayer:
-    def __init__(self, W: torch.Tensor, N: int, M: int, keep_mask: bool = False, sparse24: bool | None = None):
+    def __init__(self, W: torch.Tensor, N: int, M: int, keep_mask: bool = False, sparse24: bool = False):
         assert W.is_cuda and W.dtype == torch.bfloat16 and W.is_contiguous()
         self.W = W
         self.d_out, self.d_in = W.shape
@@ -29,8 +29,11 @@ class SparseBitLinearLayer:
         self.gamma = torch.empty(1, dtype=torch.float32, device=dev)
         self.ws_bytes = B.sbl_mask_quant_workspace_bytes(self.d_out, self.d_in)
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
-        # 2:4 weights go to the sparse tensor core through the compressed format
-        self.sparse24 = (N, M) == (2, 4) if sparse24 is None else bool(sparse24)
+        # sparse24=True sends 2:4 weights to the sparse tensor core through the
+        # compressed format.  Off by default: on B200 the dense int8 product is
+        # faster at the shapes measured (the activation tile, which sparsity
+        # does not shrink, bounds both by operand bandwidth).
+        self.sparse24 = bool(sparse24) and (N, M) == (2, 4)
         self.w24_bytes = B.sbl_compress24_bytes(self.d_out, self.d_in) if self.sparse24 else 0
         self.w24 = torch.empty(self.w24_bytes, dtype=torch.uint8, device=dev) if self.sparse24 else None
 

@@ -34,7 +34,7 @@ def _dw_rows(dy_bits, x_bits, rows, chunk=4096):
     return out
 
 
-def _run_layer_set(name, T, N=6, M=8, sample=64, seed=0):
+def _run_layer_set(name, T, N=6, M=8, sample=64, seed=0, sparse24=False):
     import semi_structured_sparsity_step_b200 as sbl
     from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer
     ls = synth.layer_set(name)
@@ -53,7 +53,7 @@ def _run_layer_set(name, T, N=6, M=8, sample=64, seed=0):
         assert np.array_equal(xq[n][toks].cpu().numpy(), rq), n
         assert np.array_equal(amax[n][toks].cpu().numpy(), ra), n
     for i, p in enumerate(ls.projections):
-        L = SparseBitLinearLayer(W[p.name].cuda(), N, M)
+        L = SparseBitLinearLayer(W[p.name].cuda(), N, M, sparse24=sparse24)
         L.weight_step()
         wb = synth.bits(W[p.name])
         weff, gamma, _ = oracle.effective_weight(wb, N, M)
@@ -98,6 +98,14 @@ def test_nm_sweep_up_proj_8192_tokens(N, M, monkeypatch):
     monkeypatch.setattr(bench, "N_KEEP", N)
     monkeypatch.setattr(bench, "M_GROUP", M)
     _run_layer_set("qwen2.5-3b-up", 8192, N=N, M=M)
+
+
+def test_2of4_sparse_tensor_core_up_proj_8192_tokens(monkeypatch):
+    """The 2:4 sweep point with the forward on the sparse tensor core
+    (sbl_compress24 + sbl_forward_sparse24), at the benchmark's size."""
+    monkeypatch.setattr(bench, "N_KEEP", 2)
+    monkeypatch.setattr(bench, "M_GROUP", 4)
+    _run_layer_set("qwen2.5-3b-up", 8192, N=2, M=4, sparse24=True)
 
 
 @pytest.mark.parametrize("batch", [1, 8, 16])
