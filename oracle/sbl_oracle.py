@@ -322,6 +322,52 @@ def unpack(packed: np.ndarray, d_out: int, d_in: int, N: int, M: int) -> np.ndar
 
 
 # --------------------------------------------------------------------------
+# Dense 2-bit ternary layout (a denser decode format)
+# [article] 7.1 推理优化技巧 (a cached low-bit format for inference).  Every
+# position keeps its 2-bit code and there is no index plane: for an N:M
+# weight the dropped positions simply hold the code of 0.  Per row, d_in / 8
+# chunks of 16 bits (little-endian halfwords, rows padded to 16 bytes); in a
+# chunk the code of position q (q < 4) sits at bits 4q..4q+1 and the code of
+# position q + 4 at bits 4q+2..4q+3 -- the chunk layout of the packed format
+# with all eight positions as slots.  Codes as above: +1 00, -1 01, 0 10.
+# --------------------------------------------------------------------------
+def dense2_row_bytes(d_in: int) -> int:
+    return _ceil16(d_in // 4)
+
+
+def pack_dense2(weff: np.ndarray) -> np.ndarray:
+    """W_eff (int8 in {-1, 0, 1}) -> dense 2-bit codes, [d_out, row bytes]."""
+    d_out, d_in = weff.shape
+    rb = dense2_row_bytes(d_in)
+    out = bytearray(d_out * rb)
+    for o in range(d_out):
+        row = bytearray(rb)
+        for pos in range(d_in):
+            c, p = divmod(pos, 8)
+            bit = 16 * c + (4 * p if p < 4 else 4 * (p - 4) + 2)
+            _put_bits(row, bit, _CODE[int(weff[o, pos])], 2)
+        out[o * rb:(o + 1) * rb] = row
+    return np.frombuffer(bytes(out), dtype=np.uint8).copy()
+
+
+def unpack_dense2(buf: np.ndarray, d_out: int, d_in: int) -> np.ndarray:
+    """Inverse of :func:`pack_dense2` (raises on the unused code 11)."""
+    rb = dense2_row_bytes(d_in)
+    assert buf.size == d_out * rb
+    data = buf.tobytes()
+    w = np.zeros((d_out, d_in), dtype=np.int8)
+    for o in range(d_out):
+        row = data[o * rb:(o + 1) * rb]
+        for pos in range(d_in):
+            c, p = divmod(pos, 8)
+            code = _get_bits(row, 16 * c + (4 * p if p < 4 else 4 * (p - 4) + 2), 2)
+            if code not in _VALUE:
+                raise ValueError(f"row {o} position {pos}: invalid code {code:#b}")
+            w[o, pos] = _VALUE[code]
+    return w
+
+
+# --------------------------------------------------------------------------
 # (a10) decode GEMV on the packed format
 # [summary] 实验结果 / Table 3 (decode on the deployed 6:8 ternary model).
 # --------------------------------------------------------------------------

@@ -384,6 +384,37 @@ def test_gemv_packed_equals_forward():
     assert np.array_equal(y, oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax))
 
 
+# ---------------------------------------------------------------- dense 2-bit layout
+def test_dense2_hand_packed_rows():
+    cases = []
+    for key, vals in _read_kv(os.path.join(GOLDEN, "dense2_rows.txt")):
+        if key == "case":
+            cases.append({})
+        else:
+            cases[-1][key] = vals
+    assert len(cases) == 2
+    for c in cases:
+        weff = np.array([int(v) for v in c["weff"]], np.int8).reshape(1, -1)
+        p = oracle.pack_dense2(weff)
+        want = np.zeros(16, np.uint8)
+        for i, b in enumerate(c["codes"]):
+            want[i] = int(b, 16)
+        assert np.array_equal(p, want), (p, want)
+        assert np.array_equal(oracle.unpack_dense2(p, 1, 8), weff)
+
+
+@pytest.mark.parametrize("N,M", [(6, 8), (2, 4), (8, 8)])
+def test_dense2_roundtrip_and_8of8_codes_plane(N, M):
+    """Round trip, and the dense layout equals the codes plane of the 8:8
+    packed format (every position a slot)."""
+    w = synth.bits(synth.trimodal_weight(5, 96, seed=16))
+    weff, _, _ = oracle.effective_weight(w, N, M)
+    d = oracle.pack_dense2(weff)
+    assert np.array_equal(oracle.unpack_dense2(d, 5, 96), weff)
+    crow, _, _ = oracle.packed_layout(5, 96, 8, 8)
+    assert np.array_equal(d, oracle.pack(weff, 8, 8)[:5 * crow])
+
+
 # ---------------------------------------------------------------- 2:4 sparse operand (a8)
 def test_sparse24_hand_compressed_row():
     kv = dict(_read_kv(os.path.join(GOLDEN, "sparse24_row.txt")))
