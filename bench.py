@@ -307,7 +307,7 @@ def run_decode(args):
     # Distinct random ternary 6:8 weights per layer, packed on the device: the
     # weight side (mask_quant) runs once per projection on random bf16 master
     # weights drawn on the device, then sbl_pack.
-    packs = []
+    packs, dense = [], []  # the packed 6:8 format, and the dense 2-bit layout of the same weights
     for l in range(layers):
         for p in ls.projections:
             w = (torch.randn(p.d_out, p.d_in, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
@@ -317,12 +317,17 @@ def run_decode(args):
             nbytes = sbl.sbl_packed_bytes(p.d_out, p.d_in, N_KEEP, M_GROUP)
             pk = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
             sbl.sbl_pack(L.W_eff, p.d_out, p.d_in, N_KEEP, M_GROUP, pk, nbytes)
+            nb2 = sbl.sbl_dense2_bytes(p.d_out, p.d_in)
+            d2 = torch.empty(nb2, dtype=torch.uint8, device="cuda")
+            sbl.sbl_pack_dense2(L.W_eff, p.d_out, p.d_in, d2, nb2)
             packs.append((p, pk, L.gamma.clone(), nbytes))
+            dense.append((d2, nb2))
             del L, w
     sbl.sbl_check()
     torch.cuda.empty_cache()
     pk_bytes = sum(x[3] for x in packs)
-    results = {}
+    d2_bytes = sum(x[1] for x in dense)
+    results, results_d2 = {}, {}
     pkk = peaks()
     for batch in (1, 8, 16):
         xs = {}
@@ -336,53 +341,68 @@ def run_decode(args):
         stream = torch.cuda.Stream()
 
         per_layer = len(ls.projections)
-        groups = []
+        groups, groups_d2 = [], []
         for l in range(layers):
-            probs = []
-            for (p, pk, gm, _), y in zip(packs[l * per_layer:(l + 1) * per_layer],
-                                         ys[l * per_layer:(l + 1) * per_layer]):
+            probs, probs_d2 = [], []
+            sl = slice(l * per_layer, (l + 1) * per_layer)
+            for (p, pk, gm, _), (d2, _), y in zip(packs[sl], dense[sl], ys[sl]):
                 xq, am = xs[p.input_name]
                 probs.append((pk, xq, am, gm, y, p.d_in, p.d_out))
+                probs_d2.append((d2, xq, am, gm, y, p.d_in, p.d_out))
             groups.append(probs)
+            groups_d2.append(probs_d2)
 
-        def one_pass():  # one grouped launch per layer: its seven projections
-            for probs in groups:
-                sbl.sbl_gemv_packed_group(probs, batch, N_KEEP, M_GROUP, stream)
-
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                one_pass()
-        stream.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            one_pass()
-        for _ in range(args.warmup):
-            graph.replay()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        reps = max(args.steps, 5)
-        e0.record(stream)
-        with torch.cuda.stream(stream):
-            for _ in range(reps):
-                graph.replay()
-        e1.record(stream)
-        stream.synchronize()
-        sbl.sbl_check()
-        ms = e0.elapsed_time(e1) / reps
-        act_bytes = sum(batch * p.d_in + 4 * batch for (p, _, _, _) in packs)
-        out_bytes = sum(4 * batch * p.d_out for (p, _, _, _) in packs)
-        tot = pk_bytes + act_bytes + out_bytes
-        gbs = tot / (ms / 1e3) / 1e9
-        results[str(batch)] = {"ms_per_pass": ms, "bytes_per_pass": tot, "packed_bytes": pk_bytes,
-                               "achieved_gbs": gbs, "frac_hbm": gbs / pkk["hbm"],
-                               "tokens_per_s_36_layers": batch / (ms / 1e3),
-                               "gemv_launches_per_pass": layers}
-        del graph
+        for variant in ("packed", "dense2"):
+            ms = _decode_pass_ms(sbl, stream, groups if variant == "packed" else groups_d2, batch, variant, args)
+            act_bytes = sum(batch * p.d_in + 4 * batch for (p, _, _, _) in packs)
+            out_bytes = sum(4 * batch * p.d_out for (p, _, _, _) in packs)
+            wb = pk_bytes if variant == "packed" else d2_bytes
+            tot = wb + act_bytes + out_bytes
+            gbs = tot / (ms / 1e3) / 1e9
+            (results if variant == "packed" else results_d2)[str(batch)] = {
+                "ms_per_pass": ms, "bytes_per_pass": tot, "weight_bytes": wb, "achieved_gbs": gbs,
+                "frac_hbm": gbs / pkk["hbm"], "tokens_per_s_36_layers": batch / (ms / 1e3),
+                "gemv_launches_per_pass": layers}
     print(json.dumps({"metric": "Sparse-BitLinear packed decode GEMV, HBM bytes/s", "unit": "GB/s",
                       "workload": f"{layers} distinct qwen2.5-3b layer sets, packed 6:8 (2.5 bit/weight), "
-                                  f"batch 1/8/16, one grouped GEMV launch per layer (7 projections), CUDA graph per pass", "peak_hbm_gbs": pkk["hbm"],
-                      "peak_source": pkk["src"], "results": results}))
+                                  f"batch 1/8/16, one grouped GEMV launch per layer (7 projections), CUDA graph per pass",
+                      "peak_hbm_gbs": pkk["hbm"], "peak_source": pkk["src"], "results": results,
+                      "dense2": {"layout": "dense 2-bit codes of the same weights (2.0 bit/weight, no index plane)",
+                                 "results": results_d2}}))
+
+
+def _decode_pass_ms(sbl, stream, groups, batch, variant, args):
+    """ms per pass over the layer stack (one grouped GEMV launch per layer),
+    captured in a CUDA graph and replayed."""
+    def one_pass():
+        for probs in groups:
+            if variant == "packed":
+                sbl.sbl_gemv_packed_group(probs, batch, N_KEEP, M_GROUP, stream)
+            else:
+                sbl.sbl_gemv_dense2_group(probs, batch, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            one_pass()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        one_pass()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    reps = max(args.steps, 5)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            graph.replay()
+    e1.record(stream)
+    stream.synchronize()
+    sbl.sbl_check()
+    del graph
+    return e0.elapsed_time(e1) / reps
 
 
 # ----------------------------------------------------------------- prefill

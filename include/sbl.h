@@ -288,6 +288,29 @@ typedef struct {
 sbl_status sbl_gemv_packed_group(const sbl_gemv_problem* problems, int count, int batch,
                                  int N, int M, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Dense 2-bit ternary layout, a denser decode format: every position keeps
+ * its 2-bit code and there is no index plane (for an N:M weight the dropped
+ * positions hold the code of 0).  [article] 7.1 (cached low-bit format for
+ * inference).  For ternary weights it is smaller than the packed format
+ * (2.0 vs 2.5 bit/weight at 6:8: a 6:8 index costs 8 bits per chunk and
+ * saves 4 bits of codes) and decodes without a table or a scatter.
+ * Layout per row, padded to 16 bytes: d_in/8 little-endian 16-bit fields;
+ * in a field the code of position q (q < 4) sits at bits 4q..4q+1 and the
+ * code of position q+4 at bits 4q+2..4q+3 (+1 = 00, -1 = 01, 0 = 10) -- the
+ * codes plane of the 8:8 packed format.
+ *   sbl_pack_dense2:       W_eff [d_out, d_in] int8 -> out (>= sbl_dense2_bytes).
+ *   sbl_gemv_dense2_group: decode GEMV on dense buffers, as
+ *                          sbl_gemv_packed_group (problems[i].packed points at
+ *                          the dense buffer of problem i; same dependent-launch
+ *                          behaviour).
+ * ---------------------------------------------------------------------- */
+size_t sbl_dense2_bytes(int d_out, int d_in);
+sbl_status sbl_pack_dense2(const int8_t* W_eff, int d_out, int d_in, uint8_t* out,
+                           size_t out_bytes, void* stream);
+sbl_status sbl_gemv_dense2_group(const sbl_gemv_problem* problems, int count, int batch,
+                                 void* stream);
+
 #ifdef __cplusplus
 }
 #endif

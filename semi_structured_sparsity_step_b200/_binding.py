@@ -47,6 +47,9 @@ SIGNATURES = {
     "sbl_unpack": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "sbl_gemv_packed": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "sbl_gemv_packed_group": (_c_int, [ctypes.POINTER(GemvProblem), _c_int, _c_int, _c_int, _c_int, _vp]),
+    "sbl_dense2_bytes": (_c_size, [_c_int, _c_int]),
+    "sbl_pack_dense2": (_c_int, [_vp, _c_int, _c_int, _vp, _c_size, _vp]),
+    "sbl_gemv_dense2_group": (_c_int, [ctypes.POINTER(GemvProblem), _c_int, _c_int, _vp]),
 }
 
 STATUS = {
@@ -203,3 +206,19 @@ def sbl_gemv_packed_group(problems, batch, N, M, stream=None) -> None:
     for i, (pk, xq, am, gm, y, d_in, d_out) in enumerate(problems):
         arr[i] = GemvProblem(_ptr(pk), _ptr(xq), _ptr(am), _ptr(gm), _ptr(y), d_in, d_out)
     _call("sbl_gemv_packed_group", arr, len(problems), batch, N, M, _stream(stream))
+
+
+def sbl_dense2_bytes(d_out, d_in) -> int:
+    return load().sbl_dense2_bytes(d_out, d_in)
+
+
+def sbl_pack_dense2(W_eff, d_out, d_in, out, out_bytes, stream=None) -> None:
+    _call("sbl_pack_dense2", _ptr(W_eff), d_out, d_in, _ptr(out), out_bytes, _stream(stream))
+
+
+def sbl_gemv_dense2_group(problems, batch, stream=None) -> None:
+    """problems: sequence of (dense2 buffer, Xq, amax, gamma, Y, d_in, d_out)."""
+    arr = (GemvProblem * len(problems))()
+    for i, (pk, xq, am, gm, y, d_in, d_out) in enumerate(problems):
+        arr[i] = GemvProblem(_ptr(pk), _ptr(xq), _ptr(am), _ptr(gm), _ptr(y), d_in, d_out)
+    _call("sbl_gemv_dense2_group", arr, len(problems), batch, _stream(stream))

@@ -186,14 +186,17 @@ constexpr int kSelTableBytes = kSelEntries * 32 * 8;
 constexpr int kTileChunks = 256;
 constexpr int kGemvThreads = 320;  // 8 consumer warps + 1 producer warp + 1 epilogue warp
 
-template <int K>
+// D2: the dense 2-bit layout (K = 8 slots = the 8 positions, no index plane,
+// no selector table, no scatter).
+template <int K, bool D2 = false>
 struct GemvTile {
   static constexpr int CODE_ROW = kTileChunks * 2 * K / 8;  // bytes per row
-  static constexpr int INDEX_ROW = kTileChunks;              // bytes per row
+  static constexpr int INDEX_ROW = D2 ? 0 : kTileChunks;     // bytes per row
   static constexpr int BYTES = 16 * (CODE_ROW + INDEX_ROW);
+  static constexpr int TABLE = D2 ? 0 : kSelTableBytes + kSelEntries * 8;
   // as many stages as still fit two blocks per SM
-  static constexpr int STAGES = K <= 6 ? 4 : 3;
-  static constexpr int SMEM = STAGES * BYTES + kSelTableBytes + kSelEntries * 8 + 128;
+  static constexpr int STAGES = D2 ? 8 : (K <= 6 ? 4 : 3);
+  static constexpr int SMEM = STAGES * BYTES + TABLE + 128;
 };
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -201,10 +204,10 @@ __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("grid
 
 // One K tile of one consumer warp: decode this lane's 8 chunks of row g
 // (and g + 8 when TWO) from the stage and multiply them into acc.
-template <int K, int NT, bool TWO>
+template <int K, int NT, bool TWO, bool D2>
 __device__ __forceinline__ void gemv_tile(int (&acc)[2][NT][4], const uint8_t* st, const uint8_t* sel_bytes,
                                           const uint4 (&xv)[NT][4], int warp, int g, int t, uint32_t lane8) {
-  using Tl = GemvTile<K>;
+  using Tl = GemvTile<K, D2>;
   using CC = ChunkCodes<K>;
   const int coff = (warp * 32 + 8 * t) * 2 * K / 8;
   uint32_t wa[5] = {0u, 0u, 0u, 0u, 0u}, wb[5] = {0u, 0u, 0u, 0u, 0u};
@@ -224,6 +227,21 @@ __device__ __forceinline__ void gemv_tile(int (&acc)[2][NT][4], const uint8_t* s
                           *reinterpret_cast<const uint16_t*>(st + (g + 8) * Tl::CODE_ROW + coff + 2 * i))
                       << (16 * (i & 1));
     }
+  }
+  if constexpr (D2) {
+    // dense 2-bit: the decoded lo / hi words are positions 0-3 / 4-7 already
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t a0, a1 = 0u, a2, a3 = 0u;
+      CC::decode(chunk_field<K>(wa, j), a0, a2);
+      if constexpr (TWO) CC::decode(chunk_field<K>(wb, j), a1, a3);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const uint4 x = xv[n][j >> 1];
+        mma_s8_16x8x32(acc[j & 1][n], a0, a1, a2, a3, (j & 1) ? x.z : x.x, (j & 1) ? x.w : x.y);
+      }
+    }
+    return;
   }
   const uint8_t* ib = st + 16 * Tl::CODE_ROW;
   const uint2 ma = *reinterpret_cast<const uint2*>(ib + g * Tl::INDEX_ROW + warp * 32 + 8 * t);
@@ -256,10 +274,10 @@ __device__ __forceinline__ void gemv_tile(int (&acc)[2][NT][4], const uint8_t* s
 // within a unit, its K tiles.  Warp 8 (one thread) issues the TMA loads
 // Tl::STAGES tiles ahead; warps 0-7 decode and multiply; warp 9 finishes
 // the units (scale and store).
-template <int K, int NT>
+template <int K, int NT, bool D2>
 __global__ void __launch_bounds__(kGemvThreads, 2)
     gemv_packed_kernel(const __grid_constant__ GemvGroup grp, uint32_t* err) {
-  using Tl = GemvTile<K>;
+  using Tl = GemvTile<K, D2>;
   using CC = ChunkCodes<K>;
   // Every shared pointer below is derived from gsm_raw by pointer arithmetic
   // (no integer casts), so the compiler keeps them in the shared window and
@@ -267,11 +285,11 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
   extern __shared__ __align__(128) uint8_t gsm_raw[];
   uint8_t* sel_bytes = gsm_raw;                                                 // [256][32] uint2
   uint2* sel_one = reinterpret_cast<uint2*>(gsm_raw + kSelTableBytes);          // [256] uint2
-  const uint32_t ring_off = kSelTableBytes + kSelEntries * 8;
+  const uint32_t ring_off = Tl::TABLE;
   uint8_t* ring = gsm_raw + ring_off + ((128u - ((smem_u32(gsm_raw) + ring_off) & 127u)) & 127u);
   __shared__ int s_acc[2][16][16];                  // unit sums [buffer][row][token]
   __shared__ float s_scale[kGemvMaxGroup][16];      // gamma * amax_tok / 127 per problem
-  __shared__ __align__(8) uint64_t s_full[4], s_empty[4];
+  __shared__ __align__(8) uint64_t s_full[Tl::STAGES], s_empty[Tl::STAGES];
   __shared__ __align__(8) uint64_t s_accf[2], s_acce[2];
   __shared__ int s_abort;
 
@@ -296,15 +314,19 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
     // while the producer (warp 8) already streams the first tiles; named
     // barrier 1 joins only these 288 threads.
     const int tid = warp == 9 ? 256 + lane : static_cast<int>(threadIdx.x);
-    for (int i = tid; i < kSelEntries; i += 288) {
-      uint32_t s0, s1;
-      scatter_selectors(static_cast<uint32_t>(i), K, s0, s1);
-      sel_one[i] = make_uint2(s0, s1);
+    if constexpr (!D2) {
+      for (int i = tid; i < kSelEntries; i += 288) {
+        uint32_t s0, s1;
+        scatter_selectors(static_cast<uint32_t>(i), K, s0, s1);
+        sel_one[i] = make_uint2(s0, s1);
+      }
     }
     for (int i = tid; i < 2 * 16 * 16; i += 288) (&s_acc[0][0][0])[i] = 0;
     asm volatile("bar.sync 1, 288;" ::: "memory");
-    uint2* tab = reinterpret_cast<uint2*>(sel_bytes);
-    for (int i = tid; i < kSelEntries * 32; i += 288) tab[i] = sel_one[i >> 5];
+    if constexpr (!D2) {
+      uint2* tab = reinterpret_cast<uint2*>(sel_bytes);
+      for (int i = tid; i < kSelEntries * 32; i += 288) tab[i] = sel_one[i >> 5];
+    }
     asm volatile("bar.sync 1, 288;" ::: "memory");
   }
   const int total = grp.unit_start[grp.count];
@@ -333,7 +355,8 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
           uint8_t* st = ring + s * Tl::BYTES;
           mbar_arrive_expect_tx(&s_full[s], rows * (Tl::CODE_ROW + Tl::INDEX_ROW));
           tma_load_2d(st, &grp.tm_codes[pi], &s_full[s], kt * (Tl::CODE_ROW / 4), row0);
-          tma_load_2d(st + 16 * Tl::CODE_ROW, &grp.tm_index[pi], &s_full[s], kt * (Tl::INDEX_ROW / 4), row0);
+          if constexpr (!D2)
+            tma_load_2d(st + 16 * Tl::CODE_ROW, &grp.tm_index[pi], &s_full[s], kt * (Tl::INDEX_ROW / 4), row0);
         }
       }
       if (!ok) {
@@ -421,9 +444,9 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
       }
       const uint8_t* st = ring + s * Tl::BYTES;
       if (two)
-        gemv_tile<K, NT, true>(acc, st, sel_bytes, xv, warp, g, t, lane8);
+        gemv_tile<K, NT, true, D2>(acc, st, sel_bytes, xv, warp, g, t, lane8);
       else
-        gemv_tile<K, NT, false>(acc, st, sel_bytes, xv, warp, g, t, lane8);
+        gemv_tile<K, NT, false, D2>(acc, st, sel_bytes, xv, warp, g, t, lane8);
       // Free the stage only now: every value read from it has been used by the
       // decode above, so no load of this warp can still be pending when the
       // next TMA copy overwrites the stage.
@@ -448,10 +471,10 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
   }
 }
 
-template <int K>
+template <int K, bool D2 = false>
 cudaError_t launch_gemv_k(const GemvGroup& grp, int units, int num_sms, cudaStream_t stream, uint32_t* err) {
-  auto kern = grp.batch <= 8 ? gemv_packed_kernel<K, 1> : gemv_packed_kernel<K, 2>;
-  const int smem = GemvTile<K>::SMEM;
+  auto kern = grp.batch <= 8 ? gemv_packed_kernel<K, 1, D2> : gemv_packed_kernel<K, 2, D2>;
+  const int smem = GemvTile<K, D2>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -534,6 +557,34 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
   }
 }
 
+// W_eff int8 -> dense 2-bit codes: one thread per 16 output bytes (8 chunks,
+// 64 weights) of a row; bytes past d_in / 4 (row padding) are written 0.
+__global__ void __launch_bounds__(256) pack_dense2_kernel(const int8_t* __restrict__ W, int d_out, int d_in,
+                                                          long long row_bytes, uint8_t* __restrict__ out) {
+  const long long per_row = row_bytes / 16;
+  const long long total = static_cast<long long>(d_out) * per_row;
+  const int nch = d_in / 8;
+  for (long long it = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; it < total;
+       it += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(it / per_row);
+    const int c0 = static_cast<int>(it - static_cast<long long>(row) * per_row) * 8;
+    uint32_t f[4] = {0u, 0u, 0u, 0u};
+    for (int j = 0; j < 8 && c0 + j < nch; ++j) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(W + static_cast<size_t>(row) * d_in) + c0 + j);
+      uint32_t field = 0u;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const int8_t q = static_cast<int8_t>(((p < 4 ? v.x : v.y) >> (8 * (p & 3))) & 0xFFu);
+        const uint32_t code = q > 0 ? 0u : (q < 0 ? 1u : 2u);  // +1 00, -1 01, 0 10
+        field |= code << (p < 4 ? 4 * p : 4 * (p - 4) + 2);
+      }
+      f[j >> 1] |= field << (16 * (j & 1));
+    }
+    *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * row_bytes + static_cast<size_t>(c0) * 2) =
+        make_uint4(f[0], f[1], f[2], f[3]);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M, uint8_t* packed,
@@ -552,8 +603,9 @@ cudaError_t launch_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M, 
 }
 
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
-                              cudaStream_t stream, int num_sms, uint32_t* err) {
+                              cudaStream_t stream, int num_sms, uint32_t* err, bool dense2) {
   if (batch == 0 || count == 0) return cudaSuccess;
+  if (dense2) N = M = 8;    // the dense layout is the codes plane of the 8:8 format
   const int K = 8 * N / M;  // slots per 8 positions
   const int code_tile_words = kTileChunks * 2 * K / 32;
   const int index_tile_words = kTileChunks / 4;
@@ -588,14 +640,20 @@ cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch,
       grp.p[i] = p;
       grp.unit_start[i] = units;
       units += (p.d_out + p.rows - 1) / p.rows;
-      if (!make_tmap_u32(&grp.tm_codes[i], p.packed, p.crow / 4, p.d_out, p.crow, code_tile_words, p.rows) ||
-          !make_tmap_u32(&grp.tm_index[i], p.packed + static_cast<size_t>(p.d_out) * p.crow, p.irow / 4, p.d_out,
-                         p.irow, index_tile_words, p.rows))
+      if (!make_tmap_u32(&grp.tm_codes[i], p.packed, p.crow / 4, p.d_out, p.crow, code_tile_words, p.rows))
+        return cudaErrorInvalidValue;
+      if (!dense2 && !make_tmap_u32(&grp.tm_index[i], p.packed + static_cast<size_t>(p.d_out) * p.crow, p.irow / 4,
+                                    p.d_out, p.irow, index_tile_words, p.rows))
         return cudaErrorInvalidValue;
     }
     grp.unit_start[grp.count] = units;
     if (units == 0) continue;
     cudaError_t e;
+    if (dense2) {
+      e = launch_gemv_k<8, true>(grp, units, num_sms, stream, err);
+      if (e != cudaSuccess) return e;
+      continue;
+    }
     switch (K) {
       case 1: e = launch_gemv_k<1>(grp, units, num_sms, stream, err); break;
       case 2: e = launch_gemv_k<2>(grp, units, num_sms, stream, err); break;
@@ -634,6 +692,20 @@ cudaError_t launch_unpack(const uint8_t* packed, int d_out, int d_in, int N, int
   return cudaGetLastError();
 }
 
+size_t dense2_row_bytes(int d_in) { return (static_cast<size_t>(d_in) / 4 + 15) / 16 * 16; }
+
+cudaError_t launch_pack_dense2(const int8_t* W_eff, int d_out, int d_in, uint8_t* out, cudaStream_t stream,
+                               int num_sms) {
+  if (d_out == 0 || d_in == 0) return cudaSuccess;
+  const long long rb = static_cast<long long>(dense2_row_bytes(d_in));
+  const long long total = static_cast<long long>(d_out) * (rb / 16);
+  long long blocks = (total + 255) / 256;
+  const long long cap = static_cast<long long>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  pack_dense2_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(W_eff, d_out, d_in, rb, out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemv_packed(const int8_t* Xq, const float* amax, int batch, const uint8_t* packed,
                                const float* gamma, int d_in, int d_out, int N, int M, float* Y,
                                cudaStream_t stream, int num_sms, uint32_t* err) {
@@ -646,7 +718,7 @@ cudaError_t launch_gemv_packed(const int8_t* Xq, const float* amax, int batch, c
   p.Y = Y;
   p.d_in = d_in;
   p.d_out = d_out;
-  return launch_gemv_group(&p, 1, batch, N, M, stream, num_sms, err);
+  return launch_gemv_group(&p, 1, batch, N, M, stream, num_sms, err, false);
 }
 
 }  // namespace sbl

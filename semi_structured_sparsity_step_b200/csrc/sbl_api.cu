@@ -324,7 +324,47 @@ sbl_status sbl_gemv_packed_group(const sbl_gemv_problem* problems, int count, in
   DeviceInfo* d = nullptr;
   if ((st = current_device(&d)) != SBL_OK) return st;
   return from_cuda(launch_gemv_group(dev.data(), count, batch, N, M, static_cast<cudaStream_t>(stream), d->num_sms,
-                                     d->err));
+                                     d->err, false));
+}
+
+size_t sbl_dense2_bytes(int d_out, int d_in) {
+  if (check_dims(d_in, d_out) != SBL_OK) return 0;
+  return static_cast<size_t>(d_out) * dense2_row_bytes(d_in);
+}
+
+sbl_status sbl_pack_dense2(const int8_t* W_eff, int d_out, int d_in, uint8_t* out, size_t out_bytes, void* stream) {
+  sbl_status st = check_dims(d_in, d_out);
+  if (st != SBL_OK) return st;
+  if (d_out == 0 || d_in == 0) return SBL_OK;
+  if (W_eff == nullptr || out == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(W_eff) || !aligned16(out)) return SBL_ERR_ALIGN;
+  if (out_bytes < sbl_dense2_bytes(d_out, d_in)) return SBL_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  return from_cuda(launch_pack_dense2(W_eff, d_out, d_in, out, static_cast<cudaStream_t>(stream), d->num_sms));
+}
+
+sbl_status sbl_gemv_dense2_group(const sbl_gemv_problem* problems, int count, int batch, void* stream) {
+  if (count < 0 || batch < 0 || batch > 16) return SBL_ERR_SHAPE;
+  if (count == 0 || batch == 0) return SBL_OK;
+  if (problems == nullptr) return SBL_ERR_INVALID_ARG;
+  std::vector<GemvProblemDev> dev(static_cast<size_t>(count));
+  sbl_status st = SBL_OK;
+  for (int i = 0; i < count; ++i) {
+    const sbl_gemv_problem& p = problems[i];
+    if ((st = check_dims(p.d_in, p.d_out)) != SBL_OK) return st;
+    if (p.d_in == 0) return SBL_ERR_SHAPE;
+    if (p.Xq == nullptr || p.amax == nullptr || p.packed == nullptr || p.gamma == nullptr || p.Y == nullptr)
+      return SBL_ERR_INVALID_ARG;
+    if (!aligned16(p.Xq) || !aligned16(p.amax) || !aligned16(p.packed) || !aligned16(p.Y) ||
+        (reinterpret_cast<uintptr_t>(p.gamma) & 3u) != 0)
+      return SBL_ERR_ALIGN;
+    dev[i] = GemvProblemDev{p.packed, p.Xq, p.amax, p.gamma, p.Y, p.d_in, p.d_out, 0, 0, 0};
+  }
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  return from_cuda(launch_gemv_group(dev.data(), count, batch, 8, 8, static_cast<cudaStream_t>(stream), d->num_sms,
+                                     d->err, true));
 }
 
 }  // extern "C"

@@ -76,7 +76,10 @@ struct GemvProblemDev {
   int rows;           // rows per work unit (16 or 8), filled in by the launcher
 };
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
-                              cudaStream_t stream, int num_sms, uint32_t* err);
+                              cudaStream_t stream, int num_sms, uint32_t* err, bool dense2);
+size_t dense2_row_bytes(int d_in);
+cudaError_t launch_pack_dense2(const int8_t* W_eff, int d_out, int d_in, uint8_t* out, cudaStream_t stream,
+                               int num_sms);
 cudaError_t launch_gemv_packed(const int8_t* Xq, const float* amax, int batch, const uint8_t* packed,
                                const float* gamma, int d_in, int d_out, int N, int M, float* Y,
                                cudaStream_t stream, int num_sms, uint32_t* err);

@@ -318,3 +318,38 @@ def test_unpack_restores_weff(lib, d_out, d_in, N, M):
     lib.sbl_check()
     assert np.array_equal(out.cpu().numpy(), weff)
     assert np.array_equal(oracle.unpack(packed.cpu().numpy(), d_out, d_in, N, M), weff)
+
+
+@pytest.mark.parametrize("d_out,d_in,N,M", [(8, 16, 6, 8), (264, 2064, 6, 8), (136, 400, 2, 4), (40, 272, 8, 8)])
+def test_pack_dense2_bit_exact(lib, d_out, d_in, N, M):
+    w = synth.trimodal_weight(d_out, d_in, seed=80, tensor_id=d_in)
+    weff, _, _ = oracle.effective_weight(synth.bits(w), N, M)
+    nbytes = lib.sbl_dense2_bytes(d_out, d_in)
+    out = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device="cuda")
+    lib.sbl_pack_dense2(torch.from_numpy(weff).cuda(), d_out, d_in, out, nbytes)
+    lib.sbl_check()
+    assert np.array_equal(out.cpu().numpy(), oracle.pack_dense2(weff))
+
+
+@pytest.mark.parametrize("batch", [1, 5, 16])
+def test_gemv_dense2_group_matches_oracle(lib, batch):
+    """Decode GEMV on the dense 2-bit layout: one grouped launch over shapes
+    that give 16- and 8-row units and a ragged last K tile."""
+    shapes = [(264, 2048), (8, 896), (520, 11008), (136, 4864)]
+    probs, refs = [], []
+    for i, (d_out, d_in) in enumerate(shapes):
+        w = synth.trimodal_weight(d_out, d_in, seed=81, tensor_id=i)
+        weff, gamma, _ = oracle.effective_weight(synth.bits(w), 6, 8)
+        x = synth.activations(batch, d_in, seed=81, tensor_id=100 + i)
+        xq, amax = oracle.act_quant(synth.bits(x))
+        nbytes = lib.sbl_dense2_bytes(d_out, d_in)
+        d2 = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        lib.sbl_pack_dense2(torch.from_numpy(weff).cuda(), d_out, d_in, d2, nbytes)
+        Y = torch.full((batch, d_out), float("nan"), dtype=torch.float32, device="cuda")
+        g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+        probs.append((d2, torch.from_numpy(xq).cuda(), torch.from_numpy(amax).cuda(), g, Y, d_in, d_out))
+        refs.append(oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax))
+    lib.sbl_gemv_dense2_group(probs, batch)
+    lib.sbl_check()
+    for (_, _, _, _, Y, _, _), ref in zip(probs, refs):
+        assert np.array_equal(Y.cpu().numpy(), ref)
