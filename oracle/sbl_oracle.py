@@ -155,6 +155,45 @@ def act_quant(x_bits: np.ndarray):
     return xq, a
 
 
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    """fp32 values -> bf16 bit patterns, round to nearest even (finite inputs)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = (u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return r.astype(np.uint16)
+
+
+# --------------------------------------------------------------------------
+# Norm before the activation quantiser: x~ = Q_a(Norm(x))
+# [summary] Algorithm 1 step (3).  The pages do not name the norm; the
+# reading taken is RMSNorm with a per-channel gain g (the norm BitNet-style
+# layers put in front of Q_a), with the arithmetic fixed so that the int8
+# codes do not depend on a summation order:
+#   ss = sum_j x_j^2 in fp64 (each bf16 square is exact in fp32),
+#   v = fl32(ss / d + eps) (fp64 division and sum, rounded once),
+#   r = fl32(1 / fl32(sqrt(v))) (IEEE sqrt and divide in fp32),
+#   xn_j = bf16(fl32(fl32(x_j * r) * g_j)) (round to nearest even),
+# then Q_a of the bf16 row xn exactly as act_quant.
+# --------------------------------------------------------------------------
+def rms_norm(x_bits: np.ndarray, g_bits: np.ndarray, eps: float):
+    """(xn bf16 bits [T, d], r fp32 [T])."""
+    x = bf16_to_f32(x_bits)
+    g = bf16_to_f32(g_bits)
+    d = x.shape[1]
+    ss = np.square(x.astype(np.float64)).sum(axis=1)
+    v = (ss / d + float(eps)).astype(np.float32)
+    r = np.divide(np.float32(1.0), np.sqrt(v, dtype=np.float32), dtype=np.float32)
+    t = np.multiply(x, r[:, None], dtype=np.float32)
+    xn = np.multiply(t, g[None, :], dtype=np.float32)
+    return f32_to_bf16(xn), r
+
+
+def rms_norm_act_quant(x_bits: np.ndarray, g_bits: np.ndarray, eps: float):
+    """(xn bf16 bits, X_q int8, amax fp32) of x~ = Q_a(RMSNorm(x))."""
+    xn, _ = rms_norm(x_bits, g_bits, eps)
+    xq, amax = act_quant(xn)
+    return xn, xq, amax
+
+
 # --------------------------------------------------------------------------
 # (a5) forward: y = (X_q . W_eff^T) * gamma * amax / 127, int32 accumulation
 # [summary] Algorithm 1 step (6) ("y ~ s * W_eff x~", s absorbs the scales);

@@ -484,3 +484,52 @@ def test_sparse24_product_and_roundtrip_ragged():
     xq[0] = -128
     xq[1] = 127
     assert np.array_equal(oracle.forward_acc_sparse24(xq, buf, 392, 784), oracle.forward_acc(xq, weff))
+
+
+# ---------------------------------------------------------------- Norm before Q_a (NEXT: fused norm + quant)
+def test_f32_to_bf16_matches_torch():
+    rng = np.random.default_rng(21)
+    v = np.concatenate([rng.normal(0, 3, 4000).astype(np.float32),
+                        # exact halfway points between neighbouring bf16 values
+                        ((np.arange(1, 200, dtype=np.uint32) << 16) | 0x8000).view(np.float32)])
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.f32_to_bf16(v), want)
+
+
+def test_rms_norm_hand_row():
+    """x = [3, 4, 0, 0], g = 1, eps = 0: ss = 25, v = 6.25, r = 0.4;
+    xn = bf16(1.2), bf16(1.6), 0, 0 = 0x3F9A (1.203125), 0x3FCD (1.6015625);
+    Q_a: amax 1.6015625, codes rint(1.203125 * 127 / 1.6015625) = 95, 127."""
+    x = synth.bits(torch.tensor([[3.0, 4.0, 0.0, 0.0]]).to(torch.bfloat16))
+    g = synth.bits(torch.ones(4).to(torch.bfloat16))
+    xn, xq, amax = oracle.rms_norm_act_quant(x, g, 0.0)
+    assert xn.tolist() == [[0x3F9A, 0x3FCD, 0, 0]]
+    assert xq.tolist() == [[95, 127, 0, 0]]
+    assert amax.tolist() == [1.6015625]
+
+
+def test_rms_norm_matches_torch_fp64():
+    x = synth.activations(64, 896, seed=22, outlier_frac=0.01)
+    g = (torch.rand(896, generator=torch.Generator().manual_seed(5)) + 0.5).to(torch.bfloat16)
+    xn, _ = oracle.rms_norm(synth.bits(x), synth.bits(g), 1e-6)
+    ref = torch.nn.functional.rms_norm(x.double(), (896,), g.double(), eps=1e-6)
+    got = oracle.bf16_to_f32(xn).astype(np.float64)
+    # within one bf16 ulp of the fp64 result, and equal to its bf16 rounding almost everywhere
+    ulp = np.abs(ref.float().to(torch.bfloat16).float().numpy()) * 2.0 ** -7
+    assert np.all(np.abs(got - ref.numpy()) <= ulp + 1e-30)
+    assert (xn == synth.bits(ref.float().to(torch.bfloat16))).mean() > 0.99
+
+
+def test_rms_norm_special_rows():
+    g = synth.bits(torch.ones(16).to(torch.bfloat16))
+    zero = np.zeros((1, 16), np.uint16)
+    xn, xq, amax = oracle.rms_norm_act_quant(zero, g, 1e-6)
+    assert not xn.any() and not xq.any() and amax.tolist() == [np.float32(1e-5)]
+    const = synth.bits(torch.full((1, 16), -0.75).to(torch.bfloat16))
+    xn, xq, _ = oracle.rms_norm_act_quant(const, g, 0.0)
+    assert np.all(oracle.bf16_to_f32(xn) == -1.0) and np.all(xq == -127)
+    # eps = 0: scaling x by a power of two leaves xn unchanged, bit for bit
+    x = synth.bits(synth.activations(8, 64, seed=23))
+    x2 = synth.bits(torch.from_numpy(oracle.bf16_to_f32(x) * 8.0).to(torch.bfloat16))
+    assert np.array_equal(oracle.rms_norm(x, synth.bits(torch.ones(64).to(torch.bfloat16)), 0.0)[0],
+                          oracle.rms_norm(x2, synth.bits(torch.ones(64).to(torch.bfloat16)), 0.0)[0])
