@@ -495,6 +495,63 @@ def run_prefill(args):
                       "results": results}))
 
 
+# ----------------------------------------------------------------- fused norm + act quant
+def run_normquant(args):
+    """Q_a(RMSNorm(x)) on the four distinct inputs of the 3B step (attn_in,
+    o_in, mlp_in, down_in; T = 32768, X ~ N(0, 1) with 0.1% outlier channels,
+    gain ~ U(0.5, 1.5)): the fused kernel (reads X, writes Xn and Xq; and
+    without the optional Xn) against sbl_act_quant alone on the same X (reads
+    X, writes Xq).  CUDA events, inputs far larger than L2."""
+    import semi_structured_sparsity_step_b200 as sbl
+    torch.cuda.set_device(0)
+    ls = synth.layer_set("qwen2.5-3b")
+    T = args.tokens or 32768
+    g_gen = torch.Generator().manual_seed(3)
+    bufs = []
+    for j, (name, d) in enumerate(ls.inputs.items()):
+        x = synth.activations(T, d, seed=0, tensor_id=100 + j, outlier_frac=0.001).cuda()
+        g = (torch.rand(d, generator=g_gen) + 0.5).to(torch.bfloat16).cuda()
+        bufs.append((x, g, d, torch.empty(T, d, dtype=torch.bfloat16, device="cuda"),
+                     torch.empty(T, d, dtype=torch.int8, device="cuda"), torch.empty(T, dtype=torch.float32,
+                                                                                    device="cuda")))
+    stream = torch.cuda.Stream()
+
+    def pass_(variant):
+        for x, g, d, xn, xq, am in bufs:
+            if variant == "rmsnorm_act_quant":
+                sbl.sbl_rmsnorm_act_quant(x, g, 1e-6, T, d, xn, xq, am, stream)
+            elif variant == "rmsnorm_act_quant_no_xn":
+                sbl.sbl_rmsnorm_act_quant(x, g, 1e-6, T, d, None, xq, am, stream)
+            else:
+                sbl.sbl_act_quant(x, T, d, xq, am, stream)
+
+    pk = peaks()
+    out = {}
+    for fused in ("rmsnorm_act_quant", "rmsnorm_act_quant_no_xn", "act_quant"):
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                pass_(fused)
+        stream.synchronize()
+        reps = max(args.steps, 5)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                pass_(fused)
+        e1.record(stream)
+        stream.synchronize()
+        sbl.sbl_check()
+        ms = e0.elapsed_time(e1) / reps
+        elems = sum(T * d for (_, _, d, _, _, _) in bufs)
+        nbytes = elems * (5 if fused == "rmsnorm_act_quant" else 3) + 4 * T * len(bufs)
+        out[fused] = {
+            "ms_per_pass": ms, "bytes": nbytes, "gbs": nbytes / (ms / 1e3) / 1e9,
+            "frac_hbm": nbytes / (ms / 1e3) / 1e9 / pk["hbm"]}
+    print(json.dumps({"metric": "Q_a(RMSNorm(x)) fused, HBM bytes/s", "unit": "GB/s", "tokens": T,
+                      "workload": "the four distinct inputs of the qwen2.5-3b layer set", "peak_hbm_gbs": pk["hbm"],
+                      "results": out}))
+
+
 # ----------------------------------------------------------------- ranks
 def rank_env():
     """(rank, world_size, local_rank) from the torchrun environment (1 process: 0, 1, 0)."""
@@ -528,7 +585,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen2.5-3b")
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (0: the workload's default)")
-    ap.add_argument("--mode", choices=["train", "decode", "prefill"], default="train")
+    ap.add_argument("--mode", choices=["train", "decode", "prefill", "normquant"], default="train")
     ap.add_argument("--layers", type=int, default=36, help="decode mode: distinct layer sets in the stack")
     ap.add_argument("--nm", default="6:8", help="N:M of the mask (the sweep: 8:8, 6:8, 4:8, 2:8, 2:4)")
     ap.add_argument("--sparse24", action="store_true", help="2:4: forward on the sparse tensor core")
@@ -541,6 +598,9 @@ def main():
         return
     if args.mode == "prefill":
         run_prefill(args)
+        return
+    if args.mode == "normquant":
+        run_normquant(args)
         return
 
     rank, world, local_rank = rank_env()

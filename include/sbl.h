@@ -144,6 +144,22 @@ sbl_status sbl_mask_quant_noalloc(const void* W, int d_out, int d_in, int N, int
 sbl_status sbl_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* amax,
                          void* stream);
 
+/* Norm fused with the activation quantiser: x~ = Q_a(Norm(x)).
+ * [summary] Algorithm 1 step (3).  Norm is RMSNorm with a per-channel gain
+ * (the pages do not name the norm), computed so that no summation order
+ * shows in the result:
+ *   ss = sum_j x_tj^2 in fp64, v = fl32(ss / d_in + eps),
+ *   r = fl32(1 / fl32(sqrt(v))), xn_tj = bf16_rn(fl32(fl32(x_tj * r) * g_j)),
+ * then Xq and amax of the bf16 row xn exactly as sbl_act_quant.  One pass
+ * over X instead of a norm pass plus sbl_act_quant.
+ *   X    [T, d_in] bf16 in (the un-normalised activation).
+ *   g    [d_in] bf16 in (the norm's gain).   eps > 0 (fp32).
+ *   Xn   optional (NULL): [T, d_in] bf16 out, the normalised row (the X
+ *        operand of sbl_backward's dW).
+ *   Xq   [T, d_in] int8 out;  amax [T] float out. */
+sbl_status sbl_rmsnorm_act_quant(const void* X, const void* g, float eps, int T, int d_in,
+                                 void* Xn, int8_t* Xq, float* amax, void* stream);
+
 /* ------------------------------------------------------------------------
  * Forward product on int8 tensor cores (tcgen05, int32 accumulation).
  * [summary] Algorithm 1 step (6): y = s * W_eff x~, with s absorbing the

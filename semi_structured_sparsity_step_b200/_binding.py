@@ -35,6 +35,7 @@ SIGNATURES = {
     "sbl_mask_quant_noalloc_scratch_bytes": (_c_size, []),
     "sbl_mask_quant_noalloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp]),
     "sbl_act_quant": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp]),
+    "sbl_rmsnorm_act_quant": (_c_int, [_vp, _vp, ctypes.c_float, _c_int, _c_int, _vp, _vp, _vp, _vp]),
     "sbl_forward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_forward_packed": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_compress24_bytes": (_c_size, [_c_int, _c_int]),
@@ -148,6 +149,11 @@ def sbl_mask_quant_noalloc(W, d_out, d_in, N, M, W_eff, W_eff_bf16, mask_bits, g
 
 def sbl_act_quant(X, T, d_in, Xq, amax, stream=None) -> None:
     _call("sbl_act_quant", _ptr(X), T, d_in, _ptr(Xq), _ptr(amax), _stream(stream))
+
+
+def sbl_rmsnorm_act_quant(X, g, eps, T, d_in, Xn, Xq, amax, stream=None) -> None:
+    _call("sbl_rmsnorm_act_quant", _ptr(X), _ptr(g), float(eps), T, d_in, _ptr(Xn), _ptr(Xq), _ptr(amax),
+          _stream(stream))
 
 
 def sbl_forward(Xq, amax, W_eff, gamma, T, d_in, d_out, Y, acc=None, stream=None) -> None:

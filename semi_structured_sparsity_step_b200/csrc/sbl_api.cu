@@ -153,6 +153,19 @@ sbl_status sbl_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* amax
   return from_cuda(launch_act_quant(X, T, d_in, Xq, amax, static_cast<cudaStream_t>(stream), d->num_sms));
 }
 
+sbl_status sbl_rmsnorm_act_quant(const void* X, const void* g, float eps, int T, int d_in, void* Xn, int8_t* Xq,
+                                 float* amax, void* stream) {
+  if (T < 0 || d_in <= 0 || d_in % 16 != 0) return SBL_ERR_SHAPE;
+  if (T == 0) return SBL_OK;
+  if (X == nullptr || g == nullptr || Xq == nullptr || amax == nullptr || !(eps > 0.0f)) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(g) || !aligned16(Xn) || !aligned16(Xq) || !aligned16(amax)) return SBL_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  sbl_status st = current_device(&d);
+  if (st != SBL_OK) return st;
+  return from_cuda(launch_norm_act_quant(X, g, eps, T, d_in, Xn, Xq, amax, static_cast<cudaStream_t>(stream),
+                                         d->num_sms));
+}
+
 sbl_status sbl_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
                        int d_in, int d_out, float* Y, int32_t* acc, void* stream) {
   sbl_status st = check_dims(d_in, d_out);

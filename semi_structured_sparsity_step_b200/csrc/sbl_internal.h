@@ -26,6 +26,8 @@ cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, 
                               uint8_t* mask_bits, float* gamma, void* workspace, cudaStream_t stream, int num_sms);
 
 // ---- activation quantiser (act_quant.cu)
+cudaError_t launch_norm_act_quant(const void* X, const void* g, float eps, int T, int d_in, void* Xn, int8_t* Xq,
+                                  float* amax, cudaStream_t stream, int num_sms);
 cudaError_t launch_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* amax, cudaStream_t stream,
                              int num_sms);
 

@@ -353,3 +353,26 @@ def test_gemv_dense2_group_matches_oracle(lib, batch):
     lib.sbl_check()
     for (_, _, _, _, Y, _, _), ref in zip(probs, refs):
         assert np.array_equal(Y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("T,d_in", [(1, 16), (64, 896), (333, 2048), (40, 4864), (17, 11008), (9, 17408)])
+@pytest.mark.parametrize("with_xn", [True, False])
+def test_rmsnorm_act_quant_matches_oracle(lib, T, d_in, with_xn):
+    """Q_a(RMSNorm(x)) in one kernel: the normalised bf16 row, the int8
+    codes and amax bit for bit against the oracle; d_in = 17408 exercises
+    the rows longer than the register-resident part."""
+    x = synth.activations(T, d_in, seed=90, tensor_id=d_in, outlier_frac=0.01)
+    if T > 2:
+        x[1] = 0.0  # an all-zero token
+    g = (torch.rand(d_in, generator=torch.Generator().manual_seed(d_in)) + 0.5).to(torch.bfloat16)
+    eps = 1e-6
+    Xn = torch.empty(T, d_in, dtype=torch.bfloat16, device="cuda") if with_xn else None
+    Xq = torch.empty(T, d_in, dtype=torch.int8, device="cuda")
+    amax = torch.empty(T, dtype=torch.float32, device="cuda")
+    lib.sbl_rmsnorm_act_quant(x.cuda(), g.cuda(), eps, T, d_in, Xn, Xq, amax)
+    lib.sbl_check()
+    rxn, rxq, ramax = oracle.rms_norm_act_quant(synth.bits(x), synth.bits(g), eps)
+    if with_xn:
+        assert np.array_equal(synth.bits(Xn.cpu()), rxn)
+    assert np.array_equal(Xq.cpu().numpy(), rxq)
+    assert np.array_equal(amax.cpu().numpy(), ramax)
