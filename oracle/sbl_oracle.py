@@ -75,9 +75,14 @@ def nm_mask(w_bits: np.ndarray, N: int, M: int, chunk: int = 1 << 18) -> np.ndar
     Position j is kept iff rank_j < N.  This keeps exactly N per group and
     breaks ties toward the lowest index.
     """
-    d_out, d_in = w_bits.shape
+    return top_n_mask(np.abs(bf16_to_f32(w_bits)), N, M, chunk)
+
+
+def top_n_mask(mag: np.ndarray, N: int, M: int, chunk: int = 1 << 18) -> np.ndarray:
+    """The rank rule of nm_mask on any array of magnitudes [d_out, d_in]."""
+    d_out, d_in = mag.shape
     assert d_in % M == 0 and 1 <= N <= M
-    a_all = np.abs(bf16_to_f32(w_bits)).reshape(-1, M)
+    a_all = mag.reshape(-1, M)
     earlier = np.tri(M, k=-1, dtype=bool)          # earlier[j, k] = (k < j)
     keep = np.empty(a_all.shape, dtype=bool)
     for s in range(0, a_all.shape[0], chunk):
@@ -134,6 +139,27 @@ def effective_weight(w_bits: np.ndarray, N: int, M: int):
 
 
 # --------------------------------------------------------------------------
+# Ablations the pages evaluate (NEXT rank 3)
+# [summary] 核心方法 / Dual-STE (masked weights keep their gradient; the
+# ablation without it multiplies dW by the mask), [gist] 2.2 and the
+# ablation of the mask source (Pi_N:M of |W_q| instead of |W|).
+# --------------------------------------------------------------------------
+def effective_weight_mask_from_quantised(w_bits: np.ndarray, N: int, M: int):
+    """Ablation: the mask is the top-N of |W_q| (values 0 or 1) per group,
+    ties to the lowest index; returns (W_eff, gamma, keep)."""
+    gamma = absmean_gamma(w_bits)
+    wq = ternary(w_bits, gamma)
+    keep = top_n_mask(np.abs(wq.astype(np.float32)), N, M)
+    weff = np.where(keep, wq, np.int8(0)).astype(np.int8)
+    return weff, gamma, keep
+
+
+def masked_grad(dw: np.ndarray, keep: np.ndarray) -> np.ndarray:
+    """Ablation without the Dual-STE: dW (.) M (masked weights get zero)."""
+    return np.where(keep, dw, np.float32(0.0)).astype(dw.dtype)
+
+
+# --------------------------------------------------------------------------
 # (a4) per-token absmax int8 activation quantisation
 # [summary] 前置知识 ("激活值另用 absmax 量化到 8-bit 整数") and Algorithm 1
 # step (3).
@@ -168,8 +194,9 @@ def f32_to_bf16(x: np.ndarray) -> np.ndarray:
 # reading taken is RMSNorm with a per-channel gain g (the norm BitNet-style
 # layers put in front of Q_a), with the arithmetic fixed so that the int8
 # codes do not depend on a summation order:
-#   ss = sum_j x_j^2 in fp64 (each bf16 square is exact in fp32),
-#   v = fl32(ss / d + eps) (fp64 division and sum, rounded once),
+#   ss = sum_j x_j^2 in fp64 (each bf16 square is exact in fp64),
+#   v = fl32(ss / d + eps) (fp64 division and sum, rounded once; eps is the
+#       fp32 value the operator is given),
 #   r = fl32(1 / fl32(sqrt(v))) (IEEE sqrt and divide in fp32),
 #   xn_j = bf16(fl32(fl32(x_j * r) * g_j)) (round to nearest even),
 # then Q_a of the bf16 row xn exactly as act_quant.
@@ -180,7 +207,7 @@ def rms_norm(x_bits: np.ndarray, g_bits: np.ndarray, eps: float):
     g = bf16_to_f32(g_bits)
     d = x.shape[1]
     ss = np.square(x.astype(np.float64)).sum(axis=1)
-    v = (ss / d + float(eps)).astype(np.float32)
+    v = (ss / d + float(np.float32(eps))).astype(np.float32)
     r = np.divide(np.float32(1.0), np.sqrt(v, dtype=np.float32), dtype=np.float32)
     t = np.multiply(x, r[:, None], dtype=np.float32)
     xn = np.multiply(t, g[None, :], dtype=np.float32)

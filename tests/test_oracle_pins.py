@@ -533,3 +533,39 @@ def test_rms_norm_special_rows():
     x2 = synth.bits(torch.from_numpy(oracle.bf16_to_f32(x) * 8.0).to(torch.bfloat16))
     assert np.array_equal(oracle.rms_norm(x, synth.bits(torch.ones(64).to(torch.bfloat16)), 0.0)[0],
                           oracle.rms_norm(x2, synth.bits(torch.ones(64).to(torch.bfloat16)), 0.0)[0])
+
+
+# ---------------------------------------------------------------- ablations (NEXT rank 3)
+@pytest.mark.parametrize("N,M", [(6, 8), (2, 4), (4, 8)])
+def test_mask_from_quantised_keeps_nonzeros_first(N, M):
+    """Pi_N:M(|W_q|): per group the kept positions are the nonzero ternary
+    positions in ascending order, then the lowest zero positions, N in all
+    (a direct restatement, checked against the rank rule)."""
+    w = synth.bits(synth.trimodal_weight(12, 64, seed=31))
+    weff, gamma, keep = oracle.effective_weight_mask_from_quantised(w, N, M)
+    wq = oracle.ternary(w, gamma)
+    for row in range(12):
+        for g in range(64 // M):
+            grp = wq[row, g * M:(g + 1) * M]
+            order = [p for p in range(M) if grp[p] != 0] + [p for p in range(M) if grp[p] == 0]
+            want = np.zeros(M, bool)
+            want[order[:N]] = True
+            assert np.array_equal(keep[row, g * M:(g + 1) * M], want)
+    # it keeps at least as many nonzero codes as the mask from |W| does
+    weff_w, _, _ = oracle.effective_weight(w, N, M)
+    assert (weff != 0).sum() >= (weff_w != 0).sum()
+
+
+def test_masked_grad_equals_autograd_of_masked_weight():
+    """dW (.) M is the gradient of y = x (W (.) M)^T with M held constant."""
+    x = synth.activations(6, 32, seed=32)
+    dy = synth.grad_output(6, 16, seed=32)
+    w = synth.bits(synth.normal_weight(16, 32, seed=32))
+    keep = oracle.nm_mask(w, 6, 8)
+    wv = torch.from_numpy(oracle.bf16_to_f32(w).astype(np.float64)).requires_grad_(True)
+    xm = torch.from_numpy(oracle.bf16_to_f32(synth.bits(x)).astype(np.float64))
+    (xm @ (wv * torch.from_numpy(keep)).T).backward(
+        torch.from_numpy(oracle.bf16_to_f32(synth.bits(dy)).astype(np.float64)))
+    got = oracle.masked_grad(oracle.backward_dw(synth.bits(dy), synth.bits(x)), keep)
+    np.testing.assert_allclose(got, wv.grad.numpy(), rtol=1e-6, atol=1e-6)
+    assert not got[~keep].any()
