@@ -107,6 +107,27 @@ sbl_status sbl_mask_quant(const void* W, int d_out, int d_in, int N, int M,
                           float* gamma, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* The weight step with the pages' mask-source ablation ([gist] 2.2 compares
+ * the mask taken from the master weight with one taken from the ternary
+ * weight).  flags = 0 is exactly sbl_mask_quant; SBL_MASK_FROM_QUANTISED
+ * takes the mask as the top-N of |W_q| per group (ties to the lowest
+ * index: the nonzero ternary codes first, then the lowest zero positions).
+ * Other arguments as sbl_mask_quant; unknown flag bits give
+ * SBL_ERR_INVALID_ARG. */
+#define SBL_MASK_FROM_QUANTISED 1u
+sbl_status sbl_mask_quant_ex(const void* W, int d_out, int d_in, int N, int M, unsigned flags,
+                             int8_t* W_eff, void* W_eff_bf16, uint8_t* mask_bits,
+                             float* gamma, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* The ablation without the Dual-STE: dW (.) M in place, so masked weights
+ * receive no gradient.  [summary] 核心方法 (the Dual-STE keeps their
+ * gradient; the ablation removes it).
+ *   dW         [d_out, d_in] float, in place (e.g. after sbl_backward).
+ *   mask_bits  [d_out, d_in/8] uint8 from sbl_mask_quant(_ex). */
+sbl_status sbl_mask_grad(float* dW, const uint8_t* mask_bits, int d_out, int d_in,
+                         void* stream);
+
 /* ------------------------------------------------------------------------
  * sbl_mask_quant without a caller-supplied workspace.  The paper has no
  * counterpart for this call: it exists for callers that cannot allocate

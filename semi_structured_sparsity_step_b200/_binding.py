@@ -32,6 +32,9 @@ SIGNATURES = {
     "sbl_set_gemm_variant": (_c_int, [_c_int]),
     "sbl_mask_quant_workspace_bytes": (_c_size, [_c_int, _c_int]),
     "sbl_mask_quant": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
+    "sbl_mask_quant_ex": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, ctypes.c_uint, _vp, _vp, _vp, _vp, _vp, _c_size,
+                                   _vp]),
+    "sbl_mask_grad": (_c_int, [_vp, _vp, _c_int, _c_int, _vp]),
     "sbl_mask_quant_noalloc_scratch_bytes": (_c_size, []),
     "sbl_mask_quant_noalloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp]),
     "sbl_act_quant": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp]),
@@ -132,6 +135,19 @@ def sbl_mask_quant(W, d_out, d_in, N, M, W_eff, W_eff_bf16, mask_bits, gamma, wo
                    stream=None) -> None:
     _call("sbl_mask_quant", _ptr(W), d_out, d_in, N, M, _ptr(W_eff), _ptr(W_eff_bf16), _ptr(mask_bits),
           _ptr(gamma), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+SBL_MASK_FROM_QUANTISED = 1
+
+
+def sbl_mask_quant_ex(W, d_out, d_in, N, M, flags, W_eff, W_eff_bf16, mask_bits, gamma, workspace, workspace_bytes,
+                      stream=None) -> None:
+    _call("sbl_mask_quant_ex", _ptr(W), d_out, d_in, N, M, int(flags), _ptr(W_eff), _ptr(W_eff_bf16), _ptr(mask_bits),
+          _ptr(gamma), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def sbl_mask_grad(dW, mask_bits, d_out, d_in, stream=None) -> None:
+    _call("sbl_mask_grad", _ptr(dW), _ptr(mask_bits), d_out, d_in, _stream(stream))
 
 
 def sbl_mask_quant_noalloc_scratch_bytes() -> int:

@@ -308,7 +308,10 @@ __device__ __forceinline__ uint32_t keep_group(const uint32_t (&key)[M]) {
   return kept;
 }
 
-template <int M, int N>
+// FROMQ (an ablation): the mask keys use whether the ternary code is nonzero
+// instead of the magnitude, so the mask is the top-N of |W_q|, ties to the
+// lowest index.
+template <int M, int N, bool FROMQ>
 __global__ void __launch_bounds__(256) ternary_mask_kernel(const uint4* __restrict__ W, size_t n_vec,
                                                            const GammaWorkspace* __restrict__ ws,
                                                            uint2* __restrict__ w_eff,
@@ -328,7 +331,8 @@ __global__ void __launch_bounds__(256) ternary_mask_kernel(const uint4* __restri
 #pragma unroll
       for (int j = 0; j < M; ++j) {
         const int pos = g * M + j;
-        const uint32_t h = (w4[pos >> 1] >> (16 * (pos & 1))) & 0x7FFFu;
+        uint32_t h = (w4[pos >> 1] >> (16 * (pos & 1))) & 0x7FFFu;
+        if constexpr (FROMQ) h = h > thr ? 1u : 0u;  // |W_q|
         key[j] = (h << 3) | static_cast<uint32_t>(M - 1 - j);
       }
       keep |= keep_group<M, N>(key) << (g * M);
@@ -358,7 +362,7 @@ size_t mask_quant_workspace_bytes() { return sizeof(GammaWorkspace); }
 
 cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, int8_t* W_eff, void* W_eff_bf16,
                               uint8_t* mask_bits, float* gamma, void* workspace, cudaStream_t stream,
-                              int num_sms) {
+                              int num_sms, bool from_quantised) {
   const size_t n = static_cast<size_t>(d_out) * d_in;
   const size_t n_vec = n / 8;
   auto* ws = static_cast<GammaWorkspace*>(workspace);
@@ -379,8 +383,9 @@ cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, 
   const uint4* w4 = static_cast<const uint4*>(W);
   uint2* we = reinterpret_cast<uint2*>(W_eff);
   uint4* wb = static_cast<uint4*>(W_eff_bf16);
-#define SBL_TERNARY(MM, NN) \
-  ternary_mask_kernel<MM, NN><<<qb, 256, 0, stream>>>(w4, n_vec, ws, we, wb, mask_bits)
+#define SBL_TERNARY(MM, NN)                                                                   \
+  (from_quantised ? ternary_mask_kernel<MM, NN, true><<<qb, 256, 0, stream>>>(w4, n_vec, ws, we, wb, mask_bits) \
+                  : ternary_mask_kernel<MM, NN, false><<<qb, 256, 0, stream>>>(w4, n_vec, ws, we, wb, mask_bits))
   if (M == 8) {
     switch (N) {
       case 1: SBL_TERNARY(8, 1); break;
@@ -404,6 +409,43 @@ cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, 
   return cudaGetLastError();
 }
 
+}  // namespace sbl
+
+// ---------------------------------------------------------------------------
+// dW (.) M: the ablation in which masked weights receive no gradient.  One
+// thread per 8 weights (two float4 and one mask byte); HBM bound.
+namespace {
+__global__ void __launch_bounds__(256) mask_grad_kernel(float4* __restrict__ dW, const uint8_t* __restrict__ bits,
+                                                        size_t n8) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint32_t m = bits[i];
+    float4 a = dW[2 * i], b = dW[2 * i + 1];
+    a.x = (m & 1u) ? a.x : 0.0f;
+    a.y = (m & 2u) ? a.y : 0.0f;
+    a.z = (m & 4u) ? a.z : 0.0f;
+    a.w = (m & 8u) ? a.w : 0.0f;
+    b.x = (m & 16u) ? b.x : 0.0f;
+    b.y = (m & 32u) ? b.y : 0.0f;
+    b.z = (m & 64u) ? b.z : 0.0f;
+    b.w = (m & 128u) ? b.w : 0.0f;
+    dW[2 * i] = a;
+    dW[2 * i + 1] = b;
+  }
+}
+}  // namespace
+
+namespace sbl {
+cudaError_t launch_mask_grad(float* dW, const uint8_t* mask_bits, int d_out, int d_in, cudaStream_t stream,
+                             int num_sms) {
+  const size_t n8 = static_cast<size_t>(d_out) * d_in / 8;
+  if (n8 == 0) return cudaSuccess;
+  size_t blocks = (n8 + 255) / 256;
+  const size_t cap = static_cast<size_t>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  mask_grad_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(reinterpret_cast<float4*>(dW), mask_bits, n8);
+  return cudaGetLastError();
+}
 }  // namespace sbl
 
 // ---------------------------------------------------------------------------

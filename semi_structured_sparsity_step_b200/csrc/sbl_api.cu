@@ -142,6 +142,38 @@ sbl_status sbl_mask_quant(const void* W, int d_out, int d_in, int N, int M, int8
                                      static_cast<cudaStream_t>(stream), d->num_sms));
 }
 
+sbl_status sbl_mask_quant_ex(const void* W, int d_out, int d_in, int N, int M, unsigned flags, int8_t* W_eff,
+                             void* W_eff_bf16, uint8_t* mask_bits, float* gamma, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if ((flags & ~static_cast<unsigned>(SBL_MASK_FROM_QUANTISED)) != 0u) return SBL_ERR_INVALID_ARG;
+  sbl_status st = check_nm(N, M);
+  if (st != SBL_OK) return st;
+  if (W == nullptr || W_eff == nullptr || gamma == nullptr || workspace == nullptr) return SBL_ERR_INVALID_ARG;
+  if ((st = check_dims(d_in, d_out)) != SBL_OK) return st;
+  const unsigned long long n = static_cast<unsigned long long>(d_out) * static_cast<unsigned long long>(d_in);
+  if (n == 0 || n >= (1ull << 32) || d_in % M != 0) return SBL_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(W_eff) || !aligned16(W_eff_bf16) || !aligned16(mask_bits) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || (reinterpret_cast<uintptr_t>(gamma) & 3u) != 0)
+    return SBL_ERR_ALIGN;
+  if (workspace_bytes < mask_quant_workspace_bytes()) return SBL_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  return from_cuda(launch_mask_quant(W, d_out, d_in, N, M, W_eff, W_eff_bf16, mask_bits, gamma, workspace,
+                                     static_cast<cudaStream_t>(stream), d->num_sms,
+                                     (flags & SBL_MASK_FROM_QUANTISED) != 0u));
+}
+
+sbl_status sbl_mask_grad(float* dW, const uint8_t* mask_bits, int d_out, int d_in, void* stream) {
+  sbl_status st = check_dims(d_in, d_out);
+  if (st != SBL_OK) return st;
+  if (d_out == 0 || d_in == 0) return SBL_OK;
+  if (dW == nullptr || mask_bits == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(dW) || !aligned16(mask_bits)) return SBL_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  return from_cuda(launch_mask_grad(dW, mask_bits, d_out, d_in, static_cast<cudaStream_t>(stream), d->num_sms));
+}
+
 sbl_status sbl_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* amax, void* stream) {
   if (T < 0 || d_in <= 0 || d_in % 16 != 0) return SBL_ERR_SHAPE;
   if (T == 0) return SBL_OK;

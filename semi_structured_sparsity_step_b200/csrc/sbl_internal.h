@@ -22,8 +22,13 @@ struct GammaWorkspace {
 };
 
 size_t mask_quant_workspace_bytes();
+// from_quantised: the mask is the top-N of |W_q| (an ablation), else of |W|.
 cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, int8_t* W_eff, void* W_eff_bf16,
-                              uint8_t* mask_bits, float* gamma, void* workspace, cudaStream_t stream, int num_sms);
+                              uint8_t* mask_bits, float* gamma, void* workspace, cudaStream_t stream, int num_sms,
+                              bool from_quantised = false);
+// dW (.) M in place (the ablation without the Dual-STE).
+cudaError_t launch_mask_grad(float* dW, const uint8_t* mask_bits, int d_out, int d_in, cudaStream_t stream,
+                             int num_sms);
 
 // ---- activation quantiser (act_quant.cu)
 cudaError_t launch_norm_act_quant(const void* X, const void* g, float eps, int T, int d_in, void* Xn, int8_t* Xq,

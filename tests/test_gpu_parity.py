@@ -376,3 +376,43 @@ def test_rmsnorm_act_quant_matches_oracle(lib, T, d_in, with_xn):
         assert np.array_equal(synth.bits(Xn.cpu()), rxn)
     assert np.array_equal(Xq.cpu().numpy(), rxq)
     assert np.array_equal(amax.cpu().numpy(), ramax)
+
+
+@pytest.mark.parametrize("d_out,d_in,N,M", [(256, 256, 6, 8), (264, 2064, 2, 4), (40, 400, 4, 8), (8, 16, 3, 4)])
+def test_mask_from_quantised_matches_oracle(lib, d_out, d_in, N, M):
+    """Ablation: the mask from |W_q| (flags = SBL_MASK_FROM_QUANTISED) gives
+    the oracle's mask, gamma and W_eff bit for bit; flags = 0 is the default."""
+    w = synth.trimodal_weight(d_out, d_in, seed=95, tensor_id=d_in)
+    wb = synth.bits(w)
+    W = w.cuda()
+    ws_bytes = lib.sbl_mask_quant_workspace_bytes(d_out, d_in)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    for flags, ref_fn in ((lib.SBL_MASK_FROM_QUANTISED, oracle.effective_weight_mask_from_quantised),
+                          (0, oracle.effective_weight)):
+        we = torch.empty(d_out, d_in, dtype=torch.int8, device="cuda")
+        bits = torch.empty(d_out, d_in // 8, dtype=torch.uint8, device="cuda")
+        g = torch.empty(1, dtype=torch.float32, device="cuda")
+        lib.sbl_mask_quant_ex(W, d_out, d_in, N, M, flags, we, None, bits, g, ws, ws_bytes)
+        lib.sbl_check()
+        rweff, rgamma, rkeep = ref_fn(wb, N, M)
+        assert g.item() == float(rgamma)
+        assert np.array_equal(we.cpu().numpy(), rweff)
+        assert np.array_equal(_unpack_mask(bits.cpu().numpy()), rkeep)
+
+
+def test_mask_grad_zeroes_masked_positions(lib):
+    """Ablation without the Dual-STE: dW (.) M after sbl_backward, exact
+    against the unmasked GPU dW and within the backward tolerance of the
+    oracle's masked gradient."""
+    T, d_out, d_in = 96, 264, 400
+    w = synth.trimodal_weight(d_out, d_in, seed=96)
+    x = synth.activations(T, d_in, seed=96, tensor_id=1)
+    dy = synth.grad_output(T, d_out, seed=96, tensor_id=2)
+    g = Layer(lib, w, x, dy, 6, 8)
+    dw = g.dW.clone()
+    lib.sbl_mask_grad(g.dW, g.L.mask_bits, d_out, d_in)
+    lib.sbl_check()
+    keep = _unpack_mask(g.L.mask_bits.cpu().numpy())
+    assert np.array_equal(g.dW.cpu().numpy(), np.where(keep, dw.cpu().numpy(), 0.0))
+    ref = oracle.masked_grad(oracle.backward_dw(synth.bits(dy), synth.bits(x)), keep)
+    _check_bwd(g.dW.cpu().numpy(), ref, "dW (.) M")
