@@ -37,7 +37,8 @@ Readings taken where the pages are silent (each is pinned by a test):
   quantiser, RoundClip and the N:M selector; no gradient flows through gamma.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-(none is "parity unpinned").
+or, for the optimizer step, ``tests/test_oracle_adamw_pins.py`` (none is
+"parity unpinned").
 """
 from __future__ import annotations
 
@@ -563,3 +564,98 @@ def forward_acc_sparse24(xq: np.ndarray, buf: np.ndarray, d_out: int, d_in: int)
     for o in range(d_out):
         acc[:, o] = (xg[:, base, i0[o]] * vals[o, :, 0]).sum(axis=1) + (xg[:, base, i1[o]] * vals[o, :, 1]).sum(axis=1)
     return acc.astype(np.int32)
+
+
+# --------------------------------------------------------------------------
+# The optimizer step after the backward pass (AdamW on the master weight),
+# gradient-norm clipping, and the mask flip count between consecutive steps.
+# [summary] Algorithm 1 step (8) (AdamW, beta = (0.9, 0.95), eps = 1e-5,
+# weight decay 0.1, grad clip 1.0, BF16 master weight W) and 局限与改进 /
+# 独立分析的弱点 (the mask flip rate of Fig. 3b: how many mask entries change
+# from one step to the next).
+#
+# Readings (the pages give only the hyperparameters):
+# * AdamW is the decoupled-decay form with bias-corrected moments;
+# * the per-step scalars are computed in fp64 from the hyperparameters and
+#   rounded once to fp32:  alpha = lr / (1 - beta1^t),
+#   b2s = sqrt(1 - beta2^t),  decay = 1 - lr * wd,  omb1 = 1 - beta1,
+#   omb2 = 1 - beta2 (beta1, beta2, eps themselves rounded to fp32);
+# * each element is updated with IEEE fp32 operations, in this order:
+#     g  = dW * c                      (c: the clipping factor, fp32)
+#     m' = beta1 * m + omb1 * g
+#     v' = beta2 * v + (omb2 * g) * g
+#     u  = m' / (sqrt(v') / b2s + eps)
+#     w' = w * decay - alpha * u
+#   every product, sum, quotient and square root rounded to fp32 on its own;
+# * the master weight is either the bf16 W itself (the pages' "BF16 master
+#   weight"; the new W is bf16_rn(w')) or an fp32 copy W32 kept beside it
+#   (the new W32 is w' and the bf16 W becomes bf16_rn(w'));
+# * clipping is by the global L2 norm of all gradients:
+#   c = fl32(min(1, max_norm / (sqrt(S) + 1e-6))) with S the sum of squares
+#   in fp64 and the sqrt and divide in fp64;
+# * the flip count is the number of positions whose keep flag differs
+#   between the mask of W before and the mask of W after the update.
+# --------------------------------------------------------------------------
+def grad_sqnorm(*grads: np.ndarray) -> float:
+    """S = sum of g^2 over every element of every gradient, correctly
+    rounded to fp64 (each fp32 square is exact in fp64; math.fsum rounds
+    the exact sum once)."""
+    parts = [np.square(np.asarray(g, np.float32).astype(np.float64)).ravel() for g in grads]
+    return math.fsum(np.concatenate(parts)) if parts else 0.0
+
+
+def grad_clip_scale(sumsq: float, max_norm: float) -> np.float32:
+    """c = fl32(min(1, max_norm / (sqrt(S) + 1e-6))), in fp64."""
+    return np.float32(min(1.0, float(max_norm) / (math.sqrt(float(sumsq)) + 1e-6)))
+
+
+def adamw_scalars(lr: float, beta1: float, beta2: float, eps: float, weight_decay: float, step: int) -> dict:
+    """The fp32 per-step scalars of AdamW at step t = step (t >= 1)."""
+    t = int(step)
+    f = np.float32
+    return {
+        "beta1": f(beta1), "beta2": f(beta2), "eps": f(eps),
+        "omb1": f(1.0 - float(beta1)), "omb2": f(1.0 - float(beta2)),
+        "alpha": f(float(lr) / (1.0 - float(beta1) ** t)),
+        "b2s": f(math.sqrt(1.0 - float(beta2) ** t)),
+        "decay": f(1.0 - float(lr) * float(weight_decay)),
+    }
+
+
+def adamw_update(w: np.ndarray, dw: np.ndarray, m: np.ndarray, v: np.ndarray, sc: dict,
+                 clip: np.float32 = np.float32(1.0)):
+    """One AdamW update of fp32 values w with gradient dw; returns
+    (w', m', v') as fp32 arrays, each step rounded to fp32."""
+    f32 = np.float32
+    w = np.asarray(w, f32)
+    g = np.multiply(np.asarray(dw, f32), f32(clip), dtype=f32)
+    m1 = np.add(np.multiply(sc["beta1"], np.asarray(m, f32), dtype=f32),
+                np.multiply(sc["omb1"], g, dtype=f32), dtype=f32)
+    v1 = np.add(np.multiply(sc["beta2"], np.asarray(v, f32), dtype=f32),
+                np.multiply(np.multiply(sc["omb2"], g, dtype=f32), g, dtype=f32), dtype=f32)
+    den = np.add(np.divide(np.sqrt(v1, dtype=f32), sc["b2s"], dtype=f32), sc["eps"], dtype=f32)
+    u = np.divide(m1, den, dtype=f32)
+    w1 = np.subtract(np.multiply(w, sc["decay"], dtype=f32), np.multiply(sc["alpha"], u, dtype=f32), dtype=f32)
+    return w1, m1, v1
+
+
+def mask_flips(keep_before: np.ndarray, keep_after: np.ndarray) -> int:
+    """Number of positions whose keep flag changed."""
+    return int(np.count_nonzero(np.asarray(keep_before, bool) != np.asarray(keep_after, bool)))
+
+
+def adamw_weight_step(w_bits: np.ndarray, dw: np.ndarray, m: np.ndarray, v: np.ndarray, N: int, M: int,
+                      sc: dict, clip: np.float32 = np.float32(1.0), w32: np.ndarray | None = None):
+    """Algorithm 1 step (8) followed by the next step's (2), (4), (5).
+
+    Returns a dict with the new bf16 W bits, the new fp32 master (or None),
+    m', v', and the next step's W_eff, gamma and keep-mask, plus the number
+    of mask flips between the mask of the old W and that of the new W.
+    """
+    master = bf16_to_f32(w_bits) if w32 is None else np.asarray(w32, np.float32)
+    w1, m1, v1 = adamw_update(master, dw, m, v, sc, clip)
+    new_bits = f32_to_bf16(w1)
+    weff, gamma, keep = effective_weight(new_bits, N, M)
+    flips = mask_flips(nm_mask(w_bits, N, M), keep)
+    return {"w_bits": new_bits, "w32": None if w32 is None else w1, "m": m1, "v": v1,
+            "weff": weff, "gamma": gamma, "keep": keep, "flips": flips}

@@ -17,7 +17,10 @@ Distributions follow the workloads the Sparse-BitNet pages describe:
 * activations and upstream gradients ~ N(0, 1), optionally with a small
   fraction of outlier channels scaled by 10;
 * groups with exact magnitude ties placed across the top-N boundary, built
-  by construction (no ranking is computed here).
+  by construction (no ranking is computed here);
+* optimizer state for the AdamW step: fp32 weight gradients ~ N(0, g_std),
+  first moments ~ N(0, 0.3 g_std) and second moments = (g_std * |z|)^2 for
+  z ~ N(0, 1) (non-negative, of the gradients' scale), g_std = 1e-3.
 """
 from __future__ import annotations
 
@@ -33,6 +36,7 @@ __all__ = [
     "activations",
     "grad_output",
     "with_boundary_ties",
+    "optimizer_state",
     "bits",
     "from_bits",
     "Projection",
@@ -129,6 +133,18 @@ def with_boundary_ties(w: torch.Tensor, N: int, M: int, seed: int = 0, tensor_id
         out[eq_groups] = 1.5 * s * esign
     # 1.5 s, 2 s .. 3 s are rounded to bf16 once here; equal inputs stay equal.
     return out.reshape(d_out, d_in).to(torch.bfloat16)
+
+
+def optimizer_state(d_out: int, d_in: int, seed: int = 0, tensor_id: int = 400,
+                    g_std: float = 1e-3):
+    """(dW, m, v) fp32 CPU tensors [d_out, d_in] for one AdamW step: the
+    gradient ~ N(0, g_std), the first moment ~ N(0, 0.3 g_std) and the second
+    moment (g_std * z)^2 with z ~ N(0, 1)."""
+    g = gen(seed, tensor_id)
+    dw = torch.randn(d_out, d_in, generator=g, dtype=torch.float32) * g_std
+    m = torch.randn(d_out, d_in, generator=g, dtype=torch.float32) * (0.3 * g_std)
+    z = torch.randn(d_out, d_in, generator=g, dtype=torch.float32) * g_std
+    return dw, m, z * z
 
 
 def bits(t: torch.Tensor) -> np.ndarray:
