@@ -129,6 +129,61 @@ sbl_status sbl_mask_grad(float* dW, const uint8_t* mask_bits, int d_out, int d_i
                          void* stream);
 
 /* ------------------------------------------------------------------------
+ * The optimizer step, fused with the first pass of the next weight step.
+ * [summary] Algorithm 1 step (8): AdamW updates the master weight (the
+ * pages: beta = (0.9, 0.95), eps = 1e-5, weight decay 0.1, grad clip 1.0,
+ * BF16 master weight); step (2) recomputes the mask from the new W on the
+ * next step; 独立分析的弱点 names the mask flip rate (Fig. 3b).
+ *
+ * sbl_grad_sqnorm: *sumsq += sum_i dW_i^2, each square exact in fp64 and
+ *   the sum in fp64 (deterministic for a given n: fixed per-block shares,
+ *   partials added in block order).  Call once per gradient tensor on one
+ *   stream, after zeroing *sumsq, to get the global squared norm that
+ *   sbl_adamw_step clips by.
+ *   dW       [n] float (any n >= 0; n = 0 adds nothing).
+ *   sumsq    1 double (device, 8-byte aligned), read and written.
+ *   workspace as sbl_mask_quant (sbl_mask_quant_workspace_bytes, 256-byte
+ *            aligned); calls sharing one workspace must be ordered.
+ * ---------------------------------------------------------------------- */
+sbl_status sbl_grad_sqnorm(const float* dW, size_t n, double* sumsq, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* sbl_adamw_step: one AdamW update of W, then the weight step of the new W
+ * (exactly what sbl_mask_quant would give for it), in two launches; the
+ * update shares its read of W with the exact gamma pass.
+ *   Per element, IEEE fp32 operations in this order (no contraction):
+ *     g  = dW * c
+ *     m' = beta1 * m + (1 - beta1) * g
+ *     v' = beta2 * v + ((1 - beta2) * g) * g
+ *     w' = w * (1 - lr * wd) - alpha * (m' / (sqrt(v') / b2s + eps))
+ *   with alpha = lr / (1 - beta1^t), b2s = sqrt(1 - beta2^t), and every
+ *   scalar (beta1, beta2, eps, 1 - beta1, 1 - beta2, alpha, b2s,
+ *   1 - lr * wd) computed in fp64 and rounded once to fp32.
+ *   c = 1 when grad_sqnorm is NULL, else fl32(min(1, max_norm /
+ *   (sqrt(S) + 1e-6))) in fp64 with S = *grad_sqnorm (device, read).
+ *   W          [d_out, d_in] bf16, in place: the new W is bf16_rn(w').
+ *   W32        optional [d_out, d_in] float master copy, in place.  NULL:
+ *              W itself is the master (w = W); else w = W32, W32 := w'.
+ *   dW         [d_out, d_in] float in.   m, v  [d_out, d_in] float, in place.
+ *   step       t >= 1 (the update's index, for the bias corrections).
+ *   lr >= 0, 0 <= beta1, beta2 < 1, eps > 0, weight_decay >= 0,
+ *   max_norm > 0 when grad_sqnorm is given.
+ *   W_eff, W_eff_bf16, mask_bits, gamma, workspace: outputs and scratch as
+ *              sbl_mask_quant, for the new W.
+ *   flips      optional 1 unsigned long long (device, 8-byte aligned): adds
+ *              the number of positions whose keep flag differs between the
+ *              mask in mask_bits on entry (the mask of the old W, from the
+ *              previous sbl_mask_quant or sbl_adamw_step) and the mask of
+ *              the new W.  Needs mask_bits; NULL skips the count. */
+sbl_status sbl_adamw_step(void* W, float* W32, const float* dW, float* m, float* v, int d_out,
+                          int d_in, int N, int M, double lr, double beta1, double beta2,
+                          double eps, double weight_decay, long long step,
+                          const double* grad_sqnorm, double max_norm, int8_t* W_eff,
+                          void* W_eff_bf16, uint8_t* mask_bits, float* gamma,
+                          unsigned long long* flips, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* ------------------------------------------------------------------------
  * sbl_mask_quant without a caller-supplied workspace.  The paper has no
  * counterpart for this call: it exists for callers that cannot allocate
  * device memory when the weight step runs, such as processes that reserve

@@ -35,6 +35,11 @@ SIGNATURES = {
     "sbl_mask_quant_ex": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, ctypes.c_uint, _vp, _vp, _vp, _vp, _vp, _c_size,
                                    _vp]),
     "sbl_mask_grad": (_c_int, [_vp, _vp, _c_int, _c_int, _vp]),
+    "sbl_grad_sqnorm": (_c_int, [_vp, _c_size, _vp, _vp, _c_size, _vp]),
+    "sbl_adamw_step": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, ctypes.c_double,
+                                ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                ctypes.c_longlong, _vp, ctypes.c_double, _vp, _vp, _vp, _vp, _vp, _vp, _c_size,
+                                _vp]),
     "sbl_mask_quant_noalloc_scratch_bytes": (_c_size, []),
     "sbl_mask_quant_noalloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp]),
     "sbl_act_quant": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp]),
@@ -148,6 +153,19 @@ def sbl_mask_quant_ex(W, d_out, d_in, N, M, flags, W_eff, W_eff_bf16, mask_bits,
 
 def sbl_mask_grad(dW, mask_bits, d_out, d_in, stream=None) -> None:
     _call("sbl_mask_grad", _ptr(dW), _ptr(mask_bits), d_out, d_in, _stream(stream))
+
+
+def sbl_grad_sqnorm(dW, n, sumsq, workspace, workspace_bytes, stream=None) -> None:
+    _call("sbl_grad_sqnorm", _ptr(dW), int(n), _ptr(sumsq), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def sbl_adamw_step(W, W32, dW, m, v, d_out, d_in, N, M, lr, beta1, beta2, eps, weight_decay, step, grad_sqnorm,
+                   max_norm, W_eff, W_eff_bf16, mask_bits, gamma, flips, workspace, workspace_bytes,
+                   stream=None) -> None:
+    _call("sbl_adamw_step", _ptr(W), _ptr(W32), _ptr(dW), _ptr(m), _ptr(v), d_out, d_in, N, M, float(lr),
+          float(beta1), float(beta2), float(eps), float(weight_decay), int(step), _ptr(grad_sqnorm),
+          float(max_norm), _ptr(W_eff), _ptr(W_eff_bf16), _ptr(mask_bits), _ptr(gamma), _ptr(flips),
+          _ptr(workspace), workspace_bytes, _stream(stream))
 
 
 def sbl_mask_quant_noalloc_scratch_bytes() -> int:

@@ -28,7 +28,9 @@
 //      ternary code is one integer compare against that threshold.  The
 //      mask ranks the 15-bit magnitudes with the position as tie-break
 //      (lower index wins), using pairwise compares in registers.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -149,52 +151,18 @@ __device__ uint32_t zero_threshold_bits_warp(float den) {
   return thr;
 }
 
-__global__ void __launch_bounds__(kGammaThreads) gamma_reduce_kernel(const uint4* __restrict__ W, size_t n_vec,
-                                                                      size_t n_elems, GammaWorkspace* ws,
-                                                                      float* __restrict__ gamma_out) {
-  __shared__ unsigned long long sbucket[256];
-  __shared__ uint64_t swarp[kGammaThreads / 32];
-  __shared__ int s_last;
-  sbucket[threadIdx.x] = 0ull;
-  __syncthreads();
-
-  // In-window magnitudes (|w| in [2^-31, 2), bf16 pattern in [0x3000, 0x4000))
-  // are added as fp64: each is a multiple of 2^-38 below 2, so a sum of up to
-  // 512 of them stays below 2^10 and needs at most 48 significant bits --
-  // every fp64 addition is exact.  The partial sum is moved into the uint64
-  // `acc` (units of 2^-38) every 512 elements.
-  uint64_t acc = 0;
-  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-  size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
-  while (i + 3 * stride < n_vec) {
-    double dacc = 0.0;
-    for (int rep = 0; rep < 16 && i + 3 * stride < n_vec; ++rep, i += 4 * stride) {  // 16 x 32 elements
-      uint4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __ldg(W + i + u * stride);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          gamma_add_bf16_f64(w4[k] & 0xFFFFu, dacc, sbucket);
-          gamma_add_bf16_f64(w4[k] >> 16, dacc, sbucket);
-        }
-      }
-    }
-    acc += static_cast<uint64_t>(scalbn(dacc, 38));
-  }
-  for (; i < n_vec; i += stride) {
-    const uint4 v = __ldg(W + i);
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      gamma_add_bf16(w4[k] & 0xFFFFu, acc, sbucket);
-      gamma_add_bf16(w4[k] >> 16, acc, sbucket);
-    }
-  }
+// End of an exact gamma pass, called by every thread of each block (256
+// threads) once its share of W has been added: `acc` is the thread's window
+// sum (units of 2^-38), `sbucket` the block's shared exponent buckets.  The
+// block's partials go to the workspace; the last block to finish adds all
+// partials exactly (320-bit integer), writes gamma = fp32(fp64(sum) / n) and
+// the zero threshold of the ternary quantiser into the workspace.
+__device__ void gamma_block_done(uint64_t acc, unsigned long long* sbucket, GammaWorkspace* ws, size_t n_elems,
+                                 float* __restrict__ gamma_out) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  __shared__ uint64_t swarp[kGammaThreads / 32];
+  __shared__ int s_last;
   if ((threadIdx.x & 31) == 0) swarp[threadIdx.x >> 5] = acc;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -268,6 +236,51 @@ __global__ void __launch_bounds__(kGammaThreads) gamma_reduce_kernel(const uint4
     const uint32_t thr = zero_threshold_bits_warp(__fadd_rn(s_gamma, 1e-5f));
     if (threadIdx.x == 0) ws->zero_threshold = thr;
   }
+}
+
+__global__ void __launch_bounds__(kGammaThreads) gamma_reduce_kernel(const uint4* __restrict__ W, size_t n_vec,
+                                                                      size_t n_elems, GammaWorkspace* ws,
+                                                                      float* __restrict__ gamma_out) {
+  __shared__ unsigned long long sbucket[256];
+  sbucket[threadIdx.x] = 0ull;
+  __syncthreads();
+
+  // In-window magnitudes (|w| in [2^-31, 2), bf16 pattern in [0x3000, 0x4000))
+  // are added as fp64: each is a multiple of 2^-38 below 2, so a sum of up to
+  // 512 of them stays below 2^10 and needs at most 48 significant bits --
+  // every fp64 addition is exact.  The partial sum is moved into the uint64
+  // `acc` (units of 2^-38) every 512 elements.
+  uint64_t acc = 0;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  while (i + 3 * stride < n_vec) {
+    double dacc = 0.0;
+    for (int rep = 0; rep < 16 && i + 3 * stride < n_vec; ++rep, i += 4 * stride) {  // 16 x 32 elements
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldg(W + i + u * stride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          gamma_add_bf16_f64(w4[k] & 0xFFFFu, dacc, sbucket);
+          gamma_add_bf16_f64(w4[k] >> 16, dacc, sbucket);
+        }
+      }
+    }
+    acc += static_cast<uint64_t>(scalbn(dacc, 38));
+  }
+  for (; i < n_vec; i += stride) {
+    const uint4 v = __ldg(W + i);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      gamma_add_bf16(w4[k] & 0xFFFFu, acc, sbucket);
+      gamma_add_bf16(w4[k] >> 16, acc, sbucket);
+    }
+  }
+  gamma_block_done(acc, sbucket, ws, n_elems, gamma_out);
 }
 
 
@@ -356,25 +369,170 @@ __global__ void __launch_bounds__(256) ternary_mask_kernel(const uint4* __restri
   }
 }
 
+// ---------------------------------------------------------------------------
+// The optimizer step fused with the first pass of the next weight step.
+// Sparse-BitNet summary, Algorithm 1 step (8): AdamW on the bf16 master
+// weight (beta = (0.9, 0.95), eps = 1e-5, weight decay 0.1, grad clip 1.0),
+// and 独立分析的弱点 (the mask flip rate of Fig. 3b).
+//
+// One thread per 8 weights: it loads the master values (8 bf16, or 8 fp32
+// when an fp32 copy is kept), 8 fp32 gradients and both fp32 moments,
+// updates them with IEEE fp32 operations in a fixed order (no contraction):
+//   g = dW * c;  m' = b1 m + (1 - b1) g;  v' = b2 v + ((1 - b2) g) g;
+//   w' = w * (1 - lr wd) - alpha * (m' / (sqrt(v') / sqrt(1 - b2^t) + eps)),
+// alpha = lr / (1 - b1^t), stores them, rounds w' to bf16 (nearest even),
+// and from the new bf16 values adds |W'| to the exact gamma sum (the same
+// integer windows and buckets as gamma_reduce_kernel) and, when asked,
+// counts the positions whose N:M keep flag differs from the mask stored for
+// the old W.  The last block finishes gamma and the ternary threshold, so
+// the next launch is the ternary pass alone: the update and the next step's
+// gamma pass share one read of W.
+struct AdamwScalars {
+  float beta1, beta2, omb1, omb2, eps, alpha, b2s, decay;
+  double max_norm;  // clipping bound (used when a squared norm is given)
+};
+
+template <int M, int N, bool MASTER32>
+__global__ void __launch_bounds__(kGammaThreads) adamw_gamma_kernel(
+    uint4* __restrict__ W, float4* __restrict__ W32, const float4* __restrict__ dW, float4* __restrict__ m,
+    float4* __restrict__ v, const uint8_t* __restrict__ old_bits, size_t n_vec, size_t n_elems, AdamwScalars sc,
+    const double* __restrict__ sumsq, GammaWorkspace* ws, float* __restrict__ gamma_out,
+    unsigned long long* __restrict__ flips) {
+  __shared__ unsigned long long sbucket[256];
+  sbucket[threadIdx.x] = 0ull;
+  __syncthreads();
+  // clipping factor c = fl32(min(1, max_norm / (sqrt(S) + 1e-6))), in fp64
+  float c = 1.0f;
+  if (sumsq != nullptr) {
+    const double q = __ddiv_rn(sc.max_norm, __dadd_rn(__dsqrt_rn(*sumsq), 1e-6));
+    c = q < 1.0 ? __double2float_rn(q) : 1.0f;
+  }
+  uint64_t acc = 0;
+  uint32_t nflip = 0;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_vec;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float w[8], g[8], mv[8], vv[8];
+    {
+      const float4 g0 = __ldcs(dW + 2 * i), g1 = __ldcs(dW + 2 * i + 1);
+      const float4 m0 = __ldcs(m + 2 * i), m1 = __ldcs(m + 2 * i + 1);
+      const float4 v0 = __ldcs(v + 2 * i), v1 = __ldcs(v + 2 * i + 1);
+      g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w; g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
+      mv[0] = m0.x; mv[1] = m0.y; mv[2] = m0.z; mv[3] = m0.w; mv[4] = m1.x; mv[5] = m1.y; mv[6] = m1.z; mv[7] = m1.w;
+      vv[0] = v0.x; vv[1] = v0.y; vv[2] = v0.z; vv[3] = v0.w; vv[4] = v1.x; vv[5] = v1.y; vv[6] = v1.z; vv[7] = v1.w;
+      if constexpr (MASTER32) {
+        const float4 a = __ldcs(W32 + 2 * i), b = __ldcs(W32 + 2 * i + 1);
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+      } else {
+        const uint4 q = W[i];
+        const uint32_t q4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          w[2 * k] = __uint_as_float(q4[k] << 16);
+          w[2 * k + 1] = __uint_as_float(q4[k] & 0xFFFF0000u);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float gk = __fmul_rn(g[k], c);
+      mv[k] = __fadd_rn(__fmul_rn(sc.beta1, mv[k]), __fmul_rn(sc.omb1, gk));
+      vv[k] = __fadd_rn(__fmul_rn(sc.beta2, vv[k]), __fmul_rn(__fmul_rn(sc.omb2, gk), gk));
+      const float den = __fadd_rn(__fdiv_rn(__fsqrt_rn(vv[k]), sc.b2s), sc.eps);
+      w[k] = __fsub_rn(__fmul_rn(w[k], sc.decay), __fmul_rn(sc.alpha, __fdiv_rn(mv[k], den)));
+    }
+    __stcs(m + 2 * i, make_float4(mv[0], mv[1], mv[2], mv[3]));
+    __stcs(m + 2 * i + 1, make_float4(mv[4], mv[5], mv[6], mv[7]));
+    __stcs(v + 2 * i, make_float4(vv[0], vv[1], vv[2], vv[3]));
+    __stcs(v + 2 * i + 1, make_float4(vv[4], vv[5], vv[6], vv[7]));
+    if constexpr (MASTER32) {
+      __stcs(W32 + 2 * i, make_float4(w[0], w[1], w[2], w[3]));
+      __stcs(W32 + 2 * i + 1, make_float4(w[4], w[5], w[6], w[7]));
+    }
+    uint32_t nb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __nv_bfloat162 p = __floats2bfloat162_rn(w[2 * k], w[2 * k + 1]);
+      nb[k] = *reinterpret_cast<const uint32_t*>(&p);
+    }
+    W[i] = make_uint4(nb[0], nb[1], nb[2], nb[3]);  // kept in L2 for the ternary pass
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      gamma_add_bf16(nb[k] & 0xFFFFu, acc, sbucket);
+      gamma_add_bf16(nb[k] >> 16, acc, sbucket);
+    }
+    if (old_bits != nullptr) {
+      uint32_t keep = 0u;
+#pragma unroll
+      for (int gi = 0; gi < 8 / M; ++gi) {
+        uint32_t key[M];
+#pragma unroll
+        for (int j = 0; j < M; ++j) {
+          const int pos = gi * M + j;
+          const uint32_t h = (nb[pos >> 1] >> (16 * (pos & 1))) & 0x7FFFu;
+          key[j] = (h << 3) | static_cast<uint32_t>(M - 1 - j);
+        }
+        keep |= keep_group<M, N>(key) << (gi * M);
+      }
+      nflip += __popc((keep ^ static_cast<uint32_t>(old_bits[i])) & 0xFFu);
+    }
+  }
+  if (old_bits != nullptr) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nflip += __shfl_xor_sync(0xFFFFFFFFu, nflip, o);
+    if ((threadIdx.x & 31) == 0 && nflip != 0u) atomicAdd(flips, static_cast<unsigned long long>(nflip));
+  }
+  gamma_block_done(acc, sbucket, ws, n_elems, gamma_out);
+}
+
+// Sum of squares of an fp32 gradient in fp64 (each square is exact in fp64),
+// added to *sumsq.  Each block sums a fixed grid-stride share and the last
+// block adds the per-block partials in block order, so the result depends
+// only on n and the grid, not on scheduling.
+__global__ void __launch_bounds__(kGammaThreads) grad_sqnorm_kernel(const float4* __restrict__ g, size_t n4,
+                                                                    const float* __restrict__ tail, int n_tail,
+                                                                    GammaWorkspace* ws, double* sumsq) {
+  __shared__ double s_w[kGammaThreads / 32];
+  double s = 0.0;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 a = __ldcs(g + i);
+    s = fma(static_cast<double>(a.x), static_cast<double>(a.x), s);
+    s = fma(static_cast<double>(a.y), static_cast<double>(a.y), s);
+    s = fma(static_cast<double>(a.z), static_cast<double>(a.z), s);
+    s = fma(static_cast<double>(a.w), static_cast<double>(a.w), s);
+  }
+  if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < n_tail) {
+    const double t = static_cast<double>(tail[threadIdx.x]);
+    s = fma(t, t, s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = s;
+  __syncthreads();
+  double* part = reinterpret_cast<double*>(ws->block_window);
+  if (threadIdx.x == 0) {
+    double b = 0.0;
+    for (int w = 0; w < kGammaThreads / 32; ++w) b += s_w[w];
+    part[blockIdx.x] = b;
+    __threadfence();
+    if (atomicAdd(&ws->ticket, 1u) == gridDim.x - 1) {
+      __threadfence();
+      double t = 0.0;
+      for (unsigned k = 0; k < gridDim.x; ++k) t += __ldcg(part + k);
+      *sumsq += t;
+    }
+  }
+}
+
 }  // namespace
 
 size_t mask_quant_workspace_bytes() { return sizeof(GammaWorkspace); }
 
-cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, int8_t* W_eff, void* W_eff_bf16,
-                              uint8_t* mask_bits, float* gamma, void* workspace, cudaStream_t stream,
-                              int num_sms, bool from_quantised) {
-  const size_t n = static_cast<size_t>(d_out) * d_in;
-  const size_t n_vec = n / 8;
-  auto* ws = static_cast<GammaWorkspace*>(workspace);
-  cudaError_t e = cudaMemsetAsync(ws, 0, offsetof(GammaWorkspace, block_window), stream);
-  if (e != cudaSuccess) return e;
-  int blocks = static_cast<int>((n_vec + kGammaThreads - 1) / kGammaThreads);
-  if (blocks > kGammaMaxBlocks) blocks = kGammaMaxBlocks;
-  if (blocks < 1) blocks = 1;
-  (void)num_sms;
-  gamma_reduce_kernel<<<blocks, kGammaThreads, 0, stream>>>(static_cast<const uint4*>(W), n_vec, n, ws, gamma);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+// The second pass of the weight step (ternary codes, W_eff, mask) for a W
+// whose gamma pass has left its threshold in ws.
+static cudaError_t launch_ternary(const void* W, size_t n_vec, int N, int M, const GammaWorkspace* ws,
+                                  int8_t* W_eff, void* W_eff_bf16, uint8_t* mask_bits, bool from_quantised,
+                                  cudaStream_t stream, int num_sms) {
   size_t qblocks = (n_vec + 255) / 256;
   const size_t qmax = static_cast<size_t>(num_sms) * 8;
   if (qblocks > qmax) qblocks = qmax;
@@ -406,6 +564,116 @@ cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, 
     }
   }
 #undef SBL_TERNARY
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, int8_t* W_eff, void* W_eff_bf16,
+                              uint8_t* mask_bits, float* gamma, void* workspace, cudaStream_t stream,
+                              int num_sms, bool from_quantised) {
+  const size_t n = static_cast<size_t>(d_out) * d_in;
+  const size_t n_vec = n / 8;
+  auto* ws = static_cast<GammaWorkspace*>(workspace);
+  cudaError_t e = cudaMemsetAsync(ws, 0, offsetof(GammaWorkspace, block_window), stream);
+  if (e != cudaSuccess) return e;
+  int blocks = static_cast<int>((n_vec + kGammaThreads - 1) / kGammaThreads);
+  if (blocks > kGammaMaxBlocks) blocks = kGammaMaxBlocks;
+  if (blocks < 1) blocks = 1;
+  (void)num_sms;
+  gamma_reduce_kernel<<<blocks, kGammaThreads, 0, stream>>>(static_cast<const uint4*>(W), n_vec, n, ws, gamma);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_ternary(W, n_vec, N, M, ws, W_eff, W_eff_bf16, mask_bits, from_quantised, stream, num_sms);
+}
+
+// fp32 per-step scalars of AdamW, computed in fp64 from the hyperparameters
+// and rounded once each (beta^t by the C library's pow).
+static AdamwScalars adamw_scalars(const AdamwParams& p) {
+  AdamwScalars sc;
+  const double t = static_cast<double>(p.step);
+  sc.beta1 = static_cast<float>(p.beta1);
+  sc.beta2 = static_cast<float>(p.beta2);
+  sc.omb1 = static_cast<float>(1.0 - p.beta1);
+  sc.omb2 = static_cast<float>(1.0 - p.beta2);
+  sc.eps = static_cast<float>(p.eps);
+  sc.alpha = static_cast<float>(p.lr / (1.0 - std::pow(p.beta1, t)));
+  sc.b2s = static_cast<float>(std::sqrt(1.0 - std::pow(p.beta2, t)));
+  sc.decay = static_cast<float>(1.0 - p.lr * p.weight_decay);
+  sc.max_norm = p.max_norm;
+  return sc;
+}
+
+template <int M, int N>
+static void adamw_launch_mn(bool master32, unsigned blocks, cudaStream_t stream, uint4* W, float4* W32,
+                            const float4* dW, float4* m, float4* v, const uint8_t* old_bits, size_t n_vec,
+                            size_t n, const AdamwScalars& sc, const double* sumsq, GammaWorkspace* ws,
+                            float* gamma, unsigned long long* flips) {
+  if (master32)
+    adamw_gamma_kernel<M, N, true><<<blocks, kGammaThreads, 0, stream>>>(W, W32, dW, m, v, old_bits, n_vec, n, sc,
+                                                                          sumsq, ws, gamma, flips);
+  else
+    adamw_gamma_kernel<M, N, false><<<blocks, kGammaThreads, 0, stream>>>(W, W32, dW, m, v, old_bits, n_vec, n, sc,
+                                                                           sumsq, ws, gamma, flips);
+}
+
+cudaError_t launch_adamw_step(void* W, float* W32, const float* dW, float* m, float* v, int d_out, int d_in, int N,
+                              int M, const AdamwParams& hp, const double* grad_sqnorm, int8_t* W_eff,
+                              void* W_eff_bf16, uint8_t* mask_bits, float* gamma, unsigned long long* flips,
+                              void* workspace, cudaStream_t stream, int num_sms) {
+  const size_t n = static_cast<size_t>(d_out) * d_in;
+  const size_t n_vec = n / 8;
+  auto* ws = static_cast<GammaWorkspace*>(workspace);
+  cudaError_t e = cudaMemsetAsync(ws, 0, offsetof(GammaWorkspace, block_window), stream);
+  if (e != cudaSuccess) return e;
+  int blocks = static_cast<int>((n_vec + kGammaThreads - 1) / kGammaThreads);
+  if (blocks > kGammaMaxBlocks) blocks = kGammaMaxBlocks;
+  if (blocks < 1) blocks = 1;
+  const AdamwScalars sc = adamw_scalars(hp);
+  const uint8_t* old_bits = flips != nullptr ? mask_bits : nullptr;
+  auto* w4 = static_cast<uint4*>(W);
+  auto* w32 = reinterpret_cast<float4*>(W32);
+  auto* g4 = reinterpret_cast<const float4*>(dW);
+  auto* m4 = reinterpret_cast<float4*>(m);
+  auto* v4 = reinterpret_cast<float4*>(v);
+  const bool master32 = W32 != nullptr;
+  const unsigned ub = static_cast<unsigned>(blocks);
+#define SBL_ADAMW(MM, NN) \
+  adamw_launch_mn<MM, NN>(master32, ub, stream, w4, w32, g4, m4, v4, old_bits, n_vec, n, sc, grad_sqnorm, ws, gamma, flips)
+  if (M == 8) {
+    switch (N) {
+      case 1: SBL_ADAMW(8, 1); break;
+      case 2: SBL_ADAMW(8, 2); break;
+      case 3: SBL_ADAMW(8, 3); break;
+      case 4: SBL_ADAMW(8, 4); break;
+      case 5: SBL_ADAMW(8, 5); break;
+      case 6: SBL_ADAMW(8, 6); break;
+      case 7: SBL_ADAMW(8, 7); break;
+      default: SBL_ADAMW(8, 8); break;
+    }
+  } else {
+    switch (N) {
+      case 1: SBL_ADAMW(4, 1); break;
+      case 2: SBL_ADAMW(4, 2); break;
+      case 3: SBL_ADAMW(4, 3); break;
+      default: SBL_ADAMW(4, 4); break;
+    }
+  }
+#undef SBL_ADAMW
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_ternary(W, n_vec, N, M, ws, W_eff, W_eff_bf16, mask_bits, false, stream, num_sms);
+}
+
+cudaError_t launch_grad_sqnorm(const float* g, size_t n, double* sumsq, void* workspace, cudaStream_t stream) {
+  auto* ws = static_cast<GammaWorkspace*>(workspace);
+  cudaError_t e = cudaMemsetAsync(&ws->ticket, 0, sizeof(ws->ticket), stream);
+  if (e != cudaSuccess) return e;
+  const size_t n4 = n / 4;
+  const int n_tail = static_cast<int>(n - 4 * n4);
+  size_t blocks = (n4 + kGammaThreads - 1) / kGammaThreads;
+  if (blocks > static_cast<size_t>(kGammaMaxBlocks)) blocks = kGammaMaxBlocks;
+  if (blocks < 1) blocks = 1;
+  grad_sqnorm_kernel<<<static_cast<unsigned>(blocks), kGammaThreads, 0, stream>>>(
+      reinterpret_cast<const float4*>(g), n4, g + 4 * n4, n_tail, ws, sumsq);
   return cudaGetLastError();
 }
 

@@ -174,6 +174,53 @@ sbl_status sbl_mask_grad(float* dW, const uint8_t* mask_bits, int d_out, int d_i
   return from_cuda(launch_mask_grad(dW, mask_bits, d_out, d_in, static_cast<cudaStream_t>(stream), d->num_sms));
 }
 
+sbl_status sbl_grad_sqnorm(const float* dW, size_t n, double* sumsq, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (sumsq == nullptr || workspace == nullptr) return SBL_ERR_INVALID_ARG;
+  if (n == 0) return SBL_OK;
+  if (dW == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(dW) || (reinterpret_cast<uintptr_t>(sumsq) & 7u) != 0 ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return SBL_ERR_ALIGN;
+  if (workspace_bytes < mask_quant_workspace_bytes()) return SBL_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  sbl_status st = current_device(&d);
+  if (st != SBL_OK) return st;
+  return from_cuda(launch_grad_sqnorm(dW, n, sumsq, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+sbl_status sbl_adamw_step(void* W, float* W32, const float* dW, float* m, float* v, int d_out, int d_in, int N,
+                          int M, double lr, double beta1, double beta2, double eps, double weight_decay,
+                          long long step, const double* grad_sqnorm, double max_norm, int8_t* W_eff,
+                          void* W_eff_bf16, uint8_t* mask_bits, float* gamma, unsigned long long* flips,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  sbl_status st = check_nm(N, M);
+  if (st != SBL_OK) return st;
+  if (W == nullptr || dW == nullptr || m == nullptr || v == nullptr || W_eff == nullptr || gamma == nullptr ||
+      workspace == nullptr)
+    return SBL_ERR_INVALID_ARG;
+  if (flips != nullptr && mask_bits == nullptr) return SBL_ERR_INVALID_ARG;
+  // hyperparameters (written so that NaN fails every test)
+  if (!(step >= 1) || !(lr >= 0.0) || !(beta1 >= 0.0 && beta1 < 1.0) || !(beta2 >= 0.0 && beta2 < 1.0) ||
+      !(eps > 0.0) || !(weight_decay >= 0.0) || (grad_sqnorm != nullptr && !(max_norm > 0.0)))
+    return SBL_ERR_INVALID_ARG;
+  if ((st = check_dims(d_in, d_out)) != SBL_OK) return st;
+  const unsigned long long n = static_cast<unsigned long long>(d_out) * static_cast<unsigned long long>(d_in);
+  if (n == 0 || n >= (1ull << 32) || d_in % M != 0) return SBL_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(W32) || !aligned16(dW) || !aligned16(m) || !aligned16(v) || !aligned16(W_eff) ||
+      !aligned16(W_eff_bf16) || !aligned16(mask_bits) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      (reinterpret_cast<uintptr_t>(gamma) & 3u) != 0 || (reinterpret_cast<uintptr_t>(grad_sqnorm) & 7u) != 0 ||
+      (reinterpret_cast<uintptr_t>(flips) & 7u) != 0)
+    return SBL_ERR_ALIGN;
+  if (workspace_bytes < mask_quant_workspace_bytes()) return SBL_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != SBL_OK) return st;
+  const AdamwParams hp{lr, beta1, beta2, eps, weight_decay, max_norm, step};
+  return from_cuda(launch_adamw_step(W, W32, dW, m, v, d_out, d_in, N, M, hp, grad_sqnorm, W_eff, W_eff_bf16,
+                                     mask_bits, gamma, flips, workspace, static_cast<cudaStream_t>(stream),
+                                     d->num_sms));
+}
+
 sbl_status sbl_act_quant(const void* X, int T, int d_in, int8_t* Xq, float* amax, void* stream) {
   if (T < 0 || d_in <= 0 || d_in % 16 != 0) return SBL_ERR_SHAPE;
   if (T == 0) return SBL_OK;

@@ -30,6 +30,19 @@ cudaError_t launch_mask_quant(const void* W, int d_out, int d_in, int N, int M, 
 cudaError_t launch_mask_grad(float* dW, const uint8_t* mask_bits, int d_out, int d_in, cudaStream_t stream,
                              int num_sms);
 
+// The optimizer step (AdamW on the master weight) fused with the next weight
+// step's gamma pass and a mask flip count, then the ternary pass.
+struct AdamwParams {
+  double lr, beta1, beta2, eps, weight_decay, max_norm;
+  long long step;  // t >= 1
+};
+cudaError_t launch_adamw_step(void* W, float* W32, const float* dW, float* m, float* v, int d_out, int d_in, int N,
+                              int M, const AdamwParams& hp, const double* grad_sqnorm, int8_t* W_eff,
+                              void* W_eff_bf16, uint8_t* mask_bits, float* gamma, unsigned long long* flips,
+                              void* workspace, cudaStream_t stream, int num_sms);
+// *sumsq += sum of g^2 (fp64, deterministic for a given n).
+cudaError_t launch_grad_sqnorm(const float* g, size_t n, double* sumsq, void* workspace, cudaStream_t stream);
+
 // ---- activation quantiser (act_quant.cu)
 cudaError_t launch_norm_act_quant(const void* X, const void* g, float eps, int T, int d_in, void* Xn, int8_t* Xq,
                                   float* amax, cudaStream_t stream, int num_sms);

@@ -66,6 +66,28 @@ def test_host_validation_without_gpu(cl):
     # workspace and packed buffer too small
     assert cl.sbl_mask_quant(al, 8, 16, 6, 8, al, None, None, al, al * 4, 8, None) == 5
     assert cl.sbl_pack(al, 8, 16, 6, 8, al, 4, None) == 5
+    # optimizer step: bad hyperparameters, flips without a mask, misalignment
+    def adamw(step=1, lr=1e-3, b1=0.9, b2=0.95, eps=1e-5, wd=0.1, sq=None, mn=1.0, bits=al, flips=None, W32=None,
+              d_in=16, ws=1 << 20):
+        return cl.sbl_adamw_step(al, W32, al, al, al, 8, d_in, 6, 8, lr, b1, b2, eps, wd, step, sq, mn, al, None,
+                                 bits, al, flips, al * 4, ws, None)
+    assert adamw(step=0) == 1
+    assert adamw(lr=-1.0) == 1
+    assert adamw(lr=float("nan")) == 1
+    assert adamw(b1=1.0) == 1
+    assert adamw(b2=-0.1) == 1
+    assert adamw(eps=0.0) == 1
+    assert adamw(wd=-0.5) == 1
+    assert adamw(sq=al, mn=0.0) == 1
+    assert adamw(bits=None, flips=al) == 1
+    assert adamw(d_in=24) == 2
+    assert adamw(W32=al + 8) == 3
+    assert adamw(sq=al + 4) == 3
+    assert adamw(ws=8) == 5
+    assert cl.sbl_grad_sqnorm(al, 16, None, al * 4, 1 << 20, None) == 1
+    assert cl.sbl_grad_sqnorm(al + 4, 16, al, al * 4, 1 << 20, None) == 3
+    assert cl.sbl_grad_sqnorm(al, 16, al, al * 4, 8, None) == 5
+    assert cl.sbl_grad_sqnorm(None, 0, al, al * 4, 1 << 20, None) == 0
     # empty work is a no-op that needs no device
     assert cl.sbl_act_quant(al, 0, 16, al, al, None) == 0
     assert cl.sbl_forward(al, al, al, al, 0, 16, 8, al, None, None) == 0
