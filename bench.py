@@ -552,6 +552,94 @@ def run_normquant(args):
                       "results": out}))
 
 
+def run_optimizer(args):
+    """The optimizer step over the 3B layer set (7 projections, 77 M weights):
+    sbl_grad_sqnorm over every dW (the global clip norm), then one
+    sbl_adamw_step per projection (AdamW on the bf16 master weight, clip at
+    max_norm 1, the next step's exact gamma pass, the mask flip count, then
+    the ternary pass).  Also the same with an fp32 master copy.  Inputs:
+    trimodal bf16 weights, synthetic fp32 gradients and moments (synth),
+    1.3 GB or more resident, far larger than L2.  CUDA events on the
+    launching stream."""
+    import semi_structured_sparsity_step_b200 as sbl
+    torch.cuda.set_device(0)
+    ls = synth.layer_set("qwen2.5-3b")
+    N, M = N_KEEP, M_GROUP
+    projs = []
+    for i, p in enumerate(ls.projections):
+        w = make_weight(ls, i, p).cuda()
+        dw, m, v = synth.optimizer_state(p.d_out, p.d_in, seed=0, tensor_id=400 + i)
+        ws_bytes = sbl.sbl_mask_quant_workspace_bytes(p.d_out, p.d_in)
+        projs.append(dict(
+            p=p, W=w, W32=w.float(), dW=dw.cuda(), m=m.cuda(), v=v.cuda(),
+            weff=torch.empty(p.d_out, p.d_in, dtype=torch.int8, device="cuda"),
+            weff16=torch.empty(p.d_out, p.d_in, dtype=torch.bfloat16, device="cuda"),
+            bits=torch.empty(p.d_out, p.d_in // 8, dtype=torch.uint8, device="cuda"),
+            gamma=torch.empty(1, dtype=torch.float32, device="cuda"),
+            ws=torch.empty(ws_bytes, dtype=torch.uint8, device="cuda"), ws_bytes=ws_bytes))
+    stream = torch.cuda.Stream()
+    sumsq = torch.zeros(1, dtype=torch.float64, device="cuda")
+    flips = torch.zeros(1, dtype=torch.int64, device="cuda")
+    with torch.cuda.stream(stream):
+        for q in projs:
+            p = q["p"]
+            sbl.sbl_mask_quant(q["W"], p.d_out, p.d_in, N, M, q["weff"], q["weff16"], q["bits"], q["gamma"],
+                               q["ws"], q["ws_bytes"], stream)
+    n_w = sum(q["p"].d_out * q["p"].d_in for q in projs)
+    state = {"t": 1000}
+
+    def sqnorm():
+        sumsq.zero_()
+        for q in projs:
+            sbl.sbl_grad_sqnorm(q["dW"], q["dW"].numel(), sumsq, q["ws"], q["ws_bytes"], stream)
+
+    def adamw(master32):
+        state["t"] += 1
+        for q in projs:
+            p = q["p"]
+            sbl.sbl_adamw_step(q["W"], q["W32"] if master32 else None, q["dW"], q["m"], q["v"], p.d_out, p.d_in,
+                               N, M, 1e-5, 0.9, 0.95, 1e-5, 0.1, state["t"], sumsq, 1.0, q["weff"], q["weff16"],
+                               q["bits"], q["gamma"], flips, q["ws"], q["ws_bytes"], stream)
+
+    # algorithmic bytes per weight: adamw launch (W 2+2 or W32 4+4 and the bf16 W write, dW 4, m 4+4,
+    # v 4+4, old mask 1/8) + ternary pass (W 2, W_eff 1, W_eff bf16 2, mask 1/8)
+    bpw = {"grad_sqnorm": 4.0, "adamw_step_bf16_master": 24.125 + 5.125,
+           "adamw_step_fp32_master": 30.125 + 5.125}
+    fns = {"grad_sqnorm": sqnorm, "adamw_step_bf16_master": lambda: adamw(False),
+           "adamw_step_fp32_master": lambda: adamw(True)}
+    pk = peaks()
+    out = {}
+    with torch.cuda.stream(stream):
+        sqnorm()
+    for name, fn in fns.items():
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                fn()
+        stream.synchronize()
+        reps = max(args.steps, 5)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                fn()
+        e1.record(stream)
+        stream.synchronize()
+        sbl.sbl_check()
+        ms = e0.elapsed_time(e1) / reps
+        gbs = bpw[name] * n_w / (ms / 1e3) / 1e9
+        out[name] = {"ms_per_pass": ms, "bytes_per_weight": bpw[name], "gbs": gbs, "frac_hbm": gbs / pk["hbm"]}
+    flip_rate = None
+    with torch.cuda.stream(stream):
+        flips.zero_()
+        adamw(False)
+    stream.synchronize()
+    flip_rate = int(flips.item()) / n_w
+    print(json.dumps({"metric": "optimizer step (AdamW + next weight step), HBM bytes/s", "unit": "GB/s",
+                      "weights": n_w, "nm": args.nm, "lr": 1e-5,
+                      "workload": "the seven projections of the qwen2.5-3b layer set",
+                      "peak_hbm_gbs": pk["hbm"], "mask_flip_rate_one_step": flip_rate, "results": out}))
+
+
 # ----------------------------------------------------------------- ranks
 def rank_env():
     """(rank, world_size, local_rank) from the torchrun environment (1 process: 0, 1, 0)."""
@@ -585,7 +673,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen2.5-3b")
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (0: the workload's default)")
-    ap.add_argument("--mode", choices=["train", "decode", "prefill", "normquant"], default="train")
+    ap.add_argument("--mode", choices=["train", "decode", "prefill", "normquant", "optimizer"], default="train")
     ap.add_argument("--layers", type=int, default=36, help="decode mode: distinct layer sets in the stack")
     ap.add_argument("--nm", default="6:8", help="N:M of the mask (the sweep: 8:8, 6:8, 4:8, 2:8, 2:4)")
     ap.add_argument("--sparse24", action="store_true", help="2:4: forward on the sparse tensor core")
@@ -601,6 +689,9 @@ def main():
         return
     if args.mode == "normquant":
         run_normquant(args)
+        return
+    if args.mode == "optimizer":
+        run_optimizer(args)
         return
 
     rank, world, local_rank = rank_env()

@@ -492,15 +492,30 @@ __global__ void __launch_bounds__(kGammaThreads) grad_sqnorm_kernel(const float4
                                                                     const float* __restrict__ tail, int n_tail,
                                                                     GammaWorkspace* ws, double* sumsq) {
   __shared__ double s_w[kGammaThreads / 32];
-  double s = 0.0;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const float4 a = __ldcs(g + i);
-    s = fma(static_cast<double>(a.x), static_cast<double>(a.x), s);
-    s = fma(static_cast<double>(a.y), static_cast<double>(a.y), s);
-    s = fma(static_cast<double>(a.z), static_cast<double>(a.z), s);
-    s = fma(static_cast<double>(a.w), static_cast<double>(a.w), s);
+  // four independent 16-byte loads in flight per thread, two accumulators
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  double s0 = 0.0, s1 = 0.0;
+  for (; i + 3 * stride < n4; i += 4 * stride) {
+    float4 a[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = __ldcs(g + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      s0 = fma(static_cast<double>(a[u].x), static_cast<double>(a[u].x), s0);
+      s1 = fma(static_cast<double>(a[u].y), static_cast<double>(a[u].y), s1);
+      s0 = fma(static_cast<double>(a[u].z), static_cast<double>(a[u].z), s0);
+      s1 = fma(static_cast<double>(a[u].w), static_cast<double>(a[u].w), s1);
+    }
   }
+  for (; i < n4; i += stride) {
+    const float4 a = __ldcs(g + i);
+    s0 = fma(static_cast<double>(a.x), static_cast<double>(a.x), s0);
+    s1 = fma(static_cast<double>(a.y), static_cast<double>(a.y), s1);
+    s0 = fma(static_cast<double>(a.z), static_cast<double>(a.z), s0);
+    s1 = fma(static_cast<double>(a.w), static_cast<double>(a.w), s1);
+  }
+  double s = s0 + s1;
   if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < n_tail) {
     const double t = static_cast<double>(tail[threadIdx.x]);
     s = fma(t, t, s);
@@ -510,17 +525,30 @@ __global__ void __launch_bounds__(kGammaThreads) grad_sqnorm_kernel(const float4
   if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = s;
   __syncthreads();
   double* part = reinterpret_cast<double*>(ws->block_window);
+  __shared__ int s_last;
   if (threadIdx.x == 0) {
     double b = 0.0;
     for (int w = 0; w < kGammaThreads / 32; ++w) b += s_w[w];
     part[blockIdx.x] = b;
     __threadfence();
-    if (atomicAdd(&ws->ticket, 1u) == gridDim.x - 1) {
-      __threadfence();
-      double t = 0.0;
-      for (unsigned k = 0; k < gridDim.x; ++k) t += __ldcg(part + k);
-      *sumsq += t;
-    }
+    s_last = atomicAdd(&ws->ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // last block: the partials in a fixed tree (thread k takes k, k + 256, ...;
+  // then the butterfly and the warps in order), so the sum does not depend
+  // on which block finished last
+  double t = 0.0;
+  for (unsigned k = threadIdx.x; k < gridDim.x; k += blockDim.x) t += __ldcg(part + k);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+  if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = t;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double u = 0.0;
+    for (int w = 0; w < kGammaThreads / 32; ++w) u += s_w[w];
+    *sumsq += u;
   }
 }
 
