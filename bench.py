@@ -300,6 +300,7 @@ def run_decode(args):
     import semi_structured_sparsity_step_b200 as sbl
     from semi_structured_sparsity_step_b200.layer import act_quant
     torch.cuda.set_device(0)
+    sbl.sbl_set_gemv_variant(args.gemv_variant)
     ls = synth.layer_set("qwen2.5-3b")
     layers = args.layers
     g = torch.Generator(device="cuda")
@@ -366,6 +367,7 @@ def run_decode(args):
     print(json.dumps({"metric": "Sparse-BitLinear packed decode GEMV, HBM bytes/s", "unit": "GB/s",
                       "workload": f"{layers} distinct qwen2.5-3b layer sets, packed 6:8 (2.5 bit/weight), "
                                   f"batch 1/8/16, one grouped GEMV launch per layer (7 projections), CUDA graph per pass",
+                      "gemv_kernel": ["per-warp streaming", "block-wide TMA ring"][args.gemv_variant],
                       "peak_hbm_gbs": pkk["hbm"], "peak_source": pkk["src"], "results": results,
                       "dense2": {"layout": "dense 2-bit codes of the same weights (2.0 bit/weight, no index plane)",
                                  "results": results_d2}}))
@@ -675,6 +677,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (0: the workload's default)")
     ap.add_argument("--mode", choices=["train", "decode", "prefill", "normquant", "optimizer"], default="train")
     ap.add_argument("--layers", type=int, default=36, help="decode mode: distinct layer sets in the stack")
+    ap.add_argument("--gemv-variant", type=int, default=0,
+                    help="decode kernel: 0 per-warp streaming (default), 1 block-wide TMA ring")
     ap.add_argument("--nm", default="6:8", help="N:M of the mask (the sweep: 8:8, 6:8, 4:8, 2:8, 2:4)")
     ap.add_argument("--sparse24", action="store_true", help="2:4: forward on the sparse tensor core")
     args = ap.parse_args()

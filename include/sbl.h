@@ -74,6 +74,14 @@ int sbl_version(void);
  * while calls are being enqueued from other threads. */
 sbl_status sbl_set_gemm_variant(int variant);
 
+/* Select the decode GEMV kernel used by sbl_gemv_packed(_group) and
+ * sbl_gemv_dense2_group for all later calls in this process: 0 = each warp
+ * streams its own rows into registers (the default), 1 = a block-wide TMA
+ * tile ring with producer and epilogue warps.  Results are identical (exact
+ * int32 sums, the same scaling).  Same threading caveat as
+ * sbl_set_gemm_variant. */
+sbl_status sbl_set_gemv_variant(int variant);
+
 /* Synchronise `stream`, then return (and clear) the first error latched by a
  * kernel of this library on the current device since the previous check;
  * SBL_OK if none.  Also reports a pending CUDA error as SBL_ERR_CUDA. */

@@ -28,6 +28,7 @@ class GemvProblem(ctypes.Structure):
 SIGNATURES = {
     "sbl_status_string": (ctypes.c_char_p, [_c_int]),
     "sbl_version": (_c_int, []),
+    "sbl_set_gemv_variant": (_c_int, [_c_int]),
     "sbl_check": (_c_int, [_vp]),
     "sbl_set_gemm_variant": (_c_int, [_c_int]),
     "sbl_mask_quant_workspace_bytes": (_c_size, [_c_int, _c_int]),
@@ -126,6 +127,10 @@ def sbl_version() -> int:
 
 def sbl_set_gemm_variant(variant: int) -> None:
     _call("sbl_set_gemm_variant", int(variant))
+
+
+def sbl_set_gemv_variant(variant: int) -> None:
+    _call("sbl_set_gemv_variant", int(variant))
 
 
 def sbl_check(stream=None) -> None:

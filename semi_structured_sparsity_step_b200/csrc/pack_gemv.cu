@@ -353,6 +353,9 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
             break;
           }
           uint8_t* st = ring + s * Tl::BYTES;
+          // the consumers' generic-proxy reads of this stage come before the
+          // async-proxy copy that overwrites it
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           mbar_arrive_expect_tx(&s_full[s], rows * (Tl::CODE_ROW + Tl::INDEX_ROW));
           tma_load_2d(st, &grp.tm_codes[pi], &s_full[s], kt * (Tl::CODE_ROW / 4), row0);
           if constexpr (!D2)
@@ -602,9 +605,19 @@ cudaError_t launch_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M, 
   return cudaGetLastError();
 }
 
+int g_gemv_variant = 0;
+
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
                               cudaStream_t stream, int num_sms, uint32_t* err, bool dense2) {
   if (batch == 0 || count == 0) return cudaSuccess;
+  if (g_gemv_variant == 0) {
+    for (int c0 = 0; c0 < count; c0 += kGemvMaxGroup) {
+      const int cnt = (count - c0) < kGemvMaxGroup ? (count - c0) : kGemvMaxGroup;
+      const cudaError_t e = launch_gemv_direct(probs + c0, cnt, batch, N, M, stream, num_sms, err, dense2);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   if (dense2) N = M = 8;    // the dense layout is the codes plane of the 8:8 format
   const int K = 8 * N / M;  // slots per 8 positions
   const int code_tile_words = kTileChunks * 2 * K / 32;

@@ -101,6 +101,12 @@ sbl_status sbl_set_gemm_variant(int variant) {
   return SBL_OK;
 }
 
+sbl_status sbl_set_gemv_variant(int variant) {
+  if (variant != 0 && variant != 1) return SBL_ERR_INVALID_ARG;
+  g_gemv_variant = variant;
+  return SBL_OK;
+}
+
 sbl_status sbl_check(void* stream) {
   DeviceInfo* d = nullptr;
   sbl_status st = current_device(&d);

@@ -95,8 +95,13 @@ struct GemvProblemDev {
   size_t crow, irow;  // filled in by the launcher
   int rows;           // rows per work unit (16 or 8), filled in by the launcher
 };
+// Decode GEMV kernel: 0 = per-warp streaming (gemv_direct.cu, the default),
+// 1 = block-wide TMA tile ring (pack_gemv.cu).
+extern int g_gemv_variant;
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
                               cudaStream_t stream, int num_sms, uint32_t* err, bool dense2);
+cudaError_t launch_gemv_direct(const GemvProblemDev* probs, int count, int batch, int N, int M,
+                               cudaStream_t stream, int num_sms, uint32_t* err, bool dense2);
 size_t dense2_row_bytes(int d_in);
 cudaError_t launch_pack_dense2(const int8_t* W_eff, int d_out, int d_in, uint8_t* out, cudaStream_t stream,
                                int num_sms);

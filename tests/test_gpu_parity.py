@@ -214,9 +214,17 @@ def test_pack_rejects_too_many_nonzeros(lib):
     lib.sbl_check()  # the latched error was cleared
 
 
+@pytest.fixture(params=[0, 1], ids=["direct", "ring"])
+def gemv_variant(request, lib):
+    """Runs a GEMV test with each decode kernel (sbl_set_gemv_variant)."""
+    lib.sbl_set_gemv_variant(request.param)
+    yield request.param
+    lib.sbl_set_gemv_variant(0)
+
+
 @pytest.mark.parametrize("batch", [1, 3, 8, 16])
 @pytest.mark.parametrize("N,M", [(6, 8), (2, 4), (8, 8)])
-def test_gemv_packed_parity(lib, batch, N, M):
+def test_gemv_packed_parity(lib, gemv_variant, batch, N, M):
     d_out, d_in = 520, 2064
     w = synth.trimodal_weight(d_out, d_in, seed=8, tensor_id=batch)
     weff, gamma, _ = oracle.effective_weight(synth.bits(w), N, M)
@@ -252,7 +260,7 @@ def test_gamma_exact_on_log_uniform_magnitudes(lib):
 
 
 @pytest.mark.parametrize("batch", [5, 16])
-def test_gemv_group_matches_single_calls(lib, batch):
+def test_gemv_group_matches_single_calls(lib, gemv_variant, batch):
     """One grouped launch over projections of different shapes equals the
     oracle.  The long-K problems run as 8-row units, the shortest as 16-row
     units, so both unit shapes are covered, with one and two token tiles."""
@@ -332,7 +340,7 @@ def test_pack_dense2_bit_exact(lib, d_out, d_in, N, M):
 
 
 @pytest.mark.parametrize("batch", [1, 5, 16])
-def test_gemv_dense2_group_matches_oracle(lib, batch):
+def test_gemv_dense2_group_matches_oracle(lib, gemv_variant, batch):
     """Decode GEMV on the dense 2-bit layout: one grouped launch over shapes
     that give 16- and 8-row units and a ragged last K tile."""
     shapes = [(264, 2048), (8, 896), (520, 11008), (136, 4864)]
@@ -353,6 +361,53 @@ def test_gemv_dense2_group_matches_oracle(lib, batch):
     lib.sbl_check()
     for (_, _, _, _, Y, _, _), ref in zip(probs, refs):
         assert np.array_equal(Y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("N,M", [(1, 8), (3, 8), (5, 8), (7, 8), (1, 4), (3, 4), (4, 8)])
+@pytest.mark.parametrize("d_out,d_in", [(8, 16), (24, 48), (40, 2320), (136, 4368)])
+def test_gemv_every_k_and_ragged_rows(lib, gemv_variant, N, M, d_out, d_in):
+    """Every slot count K = 8N/M, rows that do not fill a 16-row block, k
+    ranges shorter than one 256-weight step or not a multiple of 64 weights,
+    and rows cut into several k slices (d_in > 2048)."""
+    if d_in % M:
+        pytest.skip("d_in must be a multiple of M")
+    batch = 3
+    w = synth.trimodal_weight(d_out, d_in, seed=82, tensor_id=d_in + N)
+    weff, gamma, _ = oracle.effective_weight(synth.bits(w), N, M)
+    x = synth.activations(batch, d_in, seed=82, tensor_id=100 + d_in)
+    xq, amax = oracle.act_quant(synth.bits(x))
+    nbytes = lib.sbl_packed_bytes(d_out, d_in, N, M)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    lib.sbl_pack(torch.from_numpy(weff).cuda(), d_out, d_in, N, M, packed, nbytes)
+    Y = torch.full((batch, d_out), float("nan"), dtype=torch.float32, device="cuda")
+    g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+    lib.sbl_gemv_packed(torch.from_numpy(xq).cuda(), torch.from_numpy(amax).cuda(), batch, packed, g, d_in, d_out,
+                        N, M, Y)
+    lib.sbl_check()
+    ref = oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax)
+    assert np.array_equal(Y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("batch", [2, 11])
+def test_gemv_many_split_rows_reuse_slots(lib, batch):
+    """Rows of 4352 weights are cut into three k slices whose partial sums
+    meet in shared-memory slots; 28416 rows give every block about a dozen
+    such row blocks, more than its eight slots, so the slots are reused."""
+    d_out, d_in = 28416, 4352
+    w = synth.normal_weight(d_out, d_in, seed=83)
+    weff, gamma, _ = oracle.effective_weight(synth.bits(w), 6, 8)
+    x = synth.activations(batch, d_in, seed=83, tensor_id=100)
+    xq, amax = oracle.act_quant(synth.bits(x))
+    nbytes = lib.sbl_packed_bytes(d_out, d_in, 6, 8)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    lib.sbl_pack(torch.from_numpy(weff).cuda(), d_out, d_in, 6, 8, packed, nbytes)
+    Y = torch.full((batch, d_out), float("nan"), dtype=torch.float32, device="cuda")
+    g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+    lib.sbl_gemv_packed(torch.from_numpy(xq).cuda(), torch.from_numpy(amax).cuda(), batch, packed, g, d_in, d_out,
+                        6, 8, Y)
+    lib.sbl_check()
+    ref = oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax)
+    assert np.array_equal(Y.cpu().numpy(), ref)
 
 
 @pytest.mark.parametrize("T,d_in", [(1, 16), (64, 896), (333, 2048), (40, 4864), (17, 11008), (9, 17408)])
