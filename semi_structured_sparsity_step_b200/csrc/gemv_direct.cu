@@ -56,13 +56,22 @@ constexpr int kDMaxGroup = 16;
 constexpr int kSelEntries = 256;
 constexpr int kSelTableBytes = kSelEntries * 32 * 8;  // one uint2 per mask and lane
 
+// A stage holds 16 rows of codes then 16 rows of slot masks.  Each row is
+// copied 16 bytes wider than the stage's own bytes (the extra bytes are the
+// start of the next stage, or zero fill past the row), so that consecutive
+// rows start in different shared-memory banks and the lanes of a warp, one
+// row per lane group, read without bank conflicts.
 template <int K, bool D2>
 struct Ring {
-  static constexpr int CODE_ROW = kStageChunks * 2 * K / 8;  // bytes per row and stage (16K)
+  static constexpr int CODE_ROW = kStageChunks * 2 * K / 8;  // code bytes per row and stage (32K)
   static constexpr int MASK_ROW = D2 ? 0 : kStageChunks;     // one mask byte per chunk
-  static constexpr int STAGE = 16 * (CODE_ROW + MASK_ROW);
+  static constexpr int CODE_PITCH = CODE_ROW + 16;
+  static constexpr int MASK_PITCH = D2 ? 0 : MASK_ROW + 16;
+  static constexpr int STAGE = 16 * (CODE_PITCH + MASK_PITCH);
   static constexpr int TABLE = D2 ? 0 : kSelTableBytes + kSelEntries * 8;
-  static constexpr int SMEM = TABLE + kDWarps * kRing * STAGE + 128;
+  // warps per block: as many as fit (the 8:8 format's rings need one fewer)
+  static constexpr int WARPS = (TABLE + kDWarps * kRing * STAGE + 128 + 16384 <= 232448) ? kDWarps : kDWarps - 1;
+  static constexpr int SMEM = TABLE + WARPS * kRing * STAGE + 128;
 };
 
 struct DirectProblem {
@@ -211,8 +220,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
     s_stages[threadIdx.x] = grp.p[threadIdx.x].stages;
     s_slices[threadIdx.x] = grp.p[threadIdx.x].slices;
   }
-  if (threadIdx.x < kDWarps * kRing) mbar_init(&s_full[0][0] + threadIdx.x, 1);
-  for (int i = threadIdx.x; i < kSlots * 16 * 16; i += kDThreads) (&s_acc[0][0][0])[i] = 0;
+  if (threadIdx.x < R::WARPS * kRing) mbar_init(&s_full[0][0] + threadIdx.x, 1);
+  for (int i = threadIdx.x; i < kSlots * 16 * 16; i += blockDim.x) (&s_acc[0][0][0])[i] = 0;
   if (threadIdx.x < kSlots) {
     s_cnt[threadIdx.x] = 0;
     s_gen[threadIdx.x] = 0;
@@ -223,7 +232,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
   const int total_rb = s_rbs[count];
   int nloc = total_rb > static_cast<int>(blockIdx.x) ? (total_rb - 1 - static_cast<int>(blockIdx.x)) / G + 1 : 0;
   if (nloc > kMaxLocalRB) nloc = kMaxLocalRB;
-  for (int i = threadIdx.x; i < nloc; i += kDThreads) {  // one local row block per thread
+  for (int i = threadIdx.x; i < nloc; i += blockDim.x) {  // one local row block per thread
     const int u = static_cast<int>(blockIdx.x) + i * G;
     int pi = 0;
     while (pi + 1 < count && u >= s_rbs[pi + 1]) ++pi;
@@ -285,12 +294,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
       mbar_arrive_expect_tx(&full[slot], R::STAGE);
       tma_load_2d(st, &grp.tm_codes[p_si.pi], &full[slot], p_st * (R::CODE_ROW / 4), p_si.rb * 16);
       if constexpr (!D2)
-        tma_load_2d(st + 16 * R::CODE_ROW, &grp.tm_index[p_si.pi], &full[slot], p_st * (R::MASK_ROW / 4),
+        tma_load_2d(st + 16 * R::CODE_PITCH, &grp.tm_index[p_si.pi], &full[slot], p_st * (R::MASK_ROW / 4),
                     p_si.rb * 16);
     }
     ++issued;
     if (++p_st >= p_si.st1) {
-      p_sl += kDWarps;
+      p_sl += R::WARPS;
       if (p_sl < total) {
         p_si = slice_info(p_sl);
         p_st = p_si.st0;
@@ -301,14 +310,14 @@ __global__ void __launch_bounds__(kDThreads, 1)
   for (int i = 0; i < kRing; ++i) issue_next();
 
   if constexpr (!D2) {
-    for (int i = threadIdx.x; i < kSelEntries; i += kDThreads) {
+    for (int i = threadIdx.x; i < kSelEntries; i += blockDim.x) {
       uint32_t s0, s1;
       scatter_selectors(static_cast<uint32_t>(i), K, s0, s1);
       sel_one[i] = make_uint2(s0, s1);
     }
     __syncthreads();
     uint2* tab = reinterpret_cast<uint2*>(sel_bytes);
-    for (int i = threadIdx.x; i < kSelEntries * 32; i += kDThreads) tab[i] = sel_one[i >> 5];
+    for (int i = threadIdx.x; i < kSelEntries * 32; i += blockDim.x) tab[i] = sel_one[i >> 5];
     __syncthreads();
   }
   griddep_wait();  // activations, scales and outputs may belong to the previous kernel
@@ -317,7 +326,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
   const uint32_t lane8 = static_cast<uint32_t>(lane) * 8u;
   int consumed = 0;
   bool ok = true;
-  for (int sl = warp; sl < total && ok; sl += kDWarps) {
+  for (int sl = warp; sl < total && ok; sl += R::WARPS) {
     const SliceInfo si = slice_info(sl);
     const DirectProblem& P = grp.p[si.pi];
     const int8_t* xr[NT];
@@ -344,21 +353,21 @@ __global__ void __launch_bounds__(kDThreads, 1)
         break;
       }
       const uint8_t* sp = ring + slot * R::STAGE;
-      const uint8_t* mp = sp + 16 * R::CODE_ROW;
+      const uint8_t* mp = sp + 16 * R::CODE_PITCH;
 #pragma unroll
       for (int h = 0; h < kStageChunks / 32; h += 2) {
         // two k-steps' codes and masks of rows g and g + 8 into registers
         uint32_t wa0[5], wb0[5], wa1[5], wb1[5];
         uint2 ma0 = make_uint2(0u, 0u), mb0 = ma0, ma1 = ma0, mb1 = ma0;
-        read_codes<K>(wa0, sp + g * R::CODE_ROW + 2 * K * (t + 4 * h));
-        read_codes<K>(wb0, sp + (g + 8) * R::CODE_ROW + 2 * K * (t + 4 * h));
-        read_codes<K>(wa1, sp + g * R::CODE_ROW + 2 * K * (t + 4 * h + 4));
-        read_codes<K>(wb1, sp + (g + 8) * R::CODE_ROW + 2 * K * (t + 4 * h + 4));
+        read_codes<K>(wa0, sp + g * R::CODE_PITCH + 2 * K * (t + 4 * h));
+        read_codes<K>(wb0, sp + (g + 8) * R::CODE_PITCH + 2 * K * (t + 4 * h));
+        read_codes<K>(wa1, sp + g * R::CODE_PITCH + 2 * K * (t + 4 * h + 4));
+        read_codes<K>(wb1, sp + (g + 8) * R::CODE_PITCH + 2 * K * (t + 4 * h + 4));
         if constexpr (!D2) {
-          ma0 = *reinterpret_cast<const uint2*>(mp + g * R::MASK_ROW + 32 * h + 8 * t);
-          mb0 = *reinterpret_cast<const uint2*>(mp + (g + 8) * R::MASK_ROW + 32 * h + 8 * t);
-          ma1 = *reinterpret_cast<const uint2*>(mp + g * R::MASK_ROW + 32 * h + 32 + 8 * t);
-          mb1 = *reinterpret_cast<const uint2*>(mp + (g + 8) * R::MASK_ROW + 32 * h + 32 + 8 * t);
+          ma0 = *reinterpret_cast<const uint2*>(mp + g * R::MASK_PITCH + 32 * h + 8 * t);
+          mb0 = *reinterpret_cast<const uint2*>(mp + (g + 8) * R::MASK_PITCH + 32 * h + 8 * t);
+          ma1 = *reinterpret_cast<const uint2*>(mp + g * R::MASK_PITCH + 32 * h + 32 + 8 * t);
+          mb1 = *reinterpret_cast<const uint2*>(mp + (g + 8) * R::MASK_PITCH + 32 * h + 32 + 8 * t);
         }
         if (h + 2 >= kStageChunks / 32) {
           // every lane has read its last values of the stage: the slot may be
@@ -463,7 +472,7 @@ cudaError_t launch_direct_k(const DirectGroup& grp, int blocks, cudaStream_t str
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(blocks));
-  cfg.blockDim = dim3(kDThreads);
+  cfg.blockDim = dim3(Ring<K, D2>::WARPS * 32);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -481,7 +490,8 @@ cudaError_t launch_gemv_direct(const GemvProblemDev* probs, int count, int batch
   if (count <= 0 || count > kDMaxGroup || batch < 1 || batch > 16) return cudaErrorInvalidValue;
   if (dense2) N = M = 8;  // the dense layout is the codes plane of the 8:8 format
   const int K = 8 * N / M;
-  const int code_box = kStageChunks * 2 * K / 32;  // uint32 words per row and stage
+  const int code_box = (kStageChunks * 2 * K / 8 + 16) / 4;  // uint32 words per row and stage, + 16 B
+  const int mask_box = (kStageChunks + 16) / 4;
   DirectGroup grp{};
   int order[kDMaxGroup];  // longest rows first (insertion sort, stable)
   for (int i = 0; i < count; ++i) order[i] = i;
@@ -499,7 +509,7 @@ cudaError_t launch_gemv_direct(const GemvProblemDev* probs, int count, int batch
     if (!make_tmap_u32(&grp.tm_codes[i], q.packed, crow / 4, q.d_out, crow, code_box, 16))
       return cudaErrorInvalidValue;
     if (!dense2 && !make_tmap_u32(&grp.tm_index[i], q.packed + static_cast<size_t>(q.d_out) * crow, irow / 4,
-                                  q.d_out, irow, kStageChunks / 4, 16))
+                                  q.d_out, irow, mask_box, 16))
       return cudaErrorInvalidValue;
     DirectProblem& d = grp.p[i];
     d.Xq = q.Xq;
