@@ -142,24 +142,26 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_kernel(const uint4* __r
   const int tr = threadIdx.x % TPR;
   const int d = nv * 8;
 
+  // Every vector's arithmetic runs unconditionally (a vector past the end of
+  // the row is loaded as zeros: its squares are below 2^-252 and cannot move
+  // fl32(ss / d + eps), and it normalises and quantises to zeros); only the
+  // loads and stores are predicated, so the loops carry no divergent branches.
+  // Rows past T re-read row T - 1 and store nothing.
   for (long long base = static_cast<long long>(blockIdx.x) * RPB; base < T;
        base += static_cast<long long>(gridDim.x) * RPB) {
     const long long row = base + rib;
     const bool active = row < T;
-    const uint4* xr = X + row * static_cast<long long>(nv);
+    const uint4* xr = X + (active ? row : static_cast<long long>(T) - 1) * static_cast<long long>(nv);
     uint4 v[kNqVpt];
     double ss = 0.0;
 #pragma unroll
     for (int k = 0; k < kNqVpt; ++k) {
       const int idx = tr + k * TPR;
-      v[k] = make_uint4(0u, 0u, 0u, 0u);
-      if (active && idx < nv) {
-        v[k] = __ldg(xr + idx);
-        ss = sumsq8(v[k], ss);
-      }
+      v[k] = idx < nv ? __ldg(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
     }
-    if (active)
-      for (int idx = tr + kNqVpt * TPR; idx < nv; idx += TPR) ss = sumsq8(__ldg(xr + idx), ss);
+#pragma unroll
+    for (int k = 0; k < kNqVpt; ++k) ss = sumsq8(v[k], ss);
+    for (int idx = tr + kNqVpt * TPR; idx < nv; idx += TPR) ss = sumsq8(__ldg(xr + idx), ss);
     ss = row_reduce<TPR, double>(ss, s_sum, rib, false);
     const float vv = static_cast<float>(ss / static_cast<double>(d) + static_cast<double>(eps));
     const float r = __fdiv_rn(1.0f, __fsqrt_rn(vv));
@@ -168,35 +170,35 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_kernel(const uint4* __r
 #pragma unroll
     for (int k = 0; k < kNqVpt; ++k) {
       const int idx = tr + k * TPR;
-      if (active && idx < nv) {
-        v[k] = norm8(v[k], __ldg(G + idx), r);
-        mx = __vmaxu2(mx, maxmag8(v[k]));
-      }
+      const uint4 gk = idx < nv ? __ldg(G + idx) : make_uint4(0u, 0u, 0u, 0u);
+      v[k] = norm8(v[k], gk, r);
+      mx = __vmaxu2(mx, maxmag8(v[k]));
     }
-    if (active)
-      for (int idx = tr + kNqVpt * TPR; idx < nv; idx += TPR)
-        mx = __vmaxu2(mx, maxmag8(norm8(__ldg(xr + idx), __ldg(G + idx), r)));
+    for (int idx = tr + kNqVpt * TPR; idx < nv; idx += TPR)
+      mx = __vmaxu2(mx, maxmag8(norm8(__ldg(xr + idx), __ldg(G + idx), r)));
     mx = max(mx & 0xFFFFu, mx >> 16);
     mx = row_reduce<TPR, uint32_t>(mx, s_max, rib, true);
-    if (!active) continue;
     const float a = fmaxf(__uint_as_float(mx << 16), 1e-5f);
-    const float s = __fdiv_rn(127.0f, a);
+    const float sc = __fdiv_rn(127.0f, a);
     uint2* qr = Xq + row * static_cast<long long>(nv);
     uint4* nr = Xn != nullptr ? Xn + row * static_cast<long long>(nv) : nullptr;
 #pragma unroll
     for (int k = 0; k < kNqVpt; ++k) {
       const int idx = tr + k * TPR;
-      if (idx < nv) {
-        qr[idx] = quant8(v[k], s);
+      const uint2 q = quant8(v[k], sc);
+      if (active && idx < nv) {
+        qr[idx] = q;
         if (nr != nullptr) nr[idx] = v[k];
       }
     }
-    for (int idx = tr + kNqVpt * TPR; idx < nv; idx += TPR) {
-      const uint4 u = norm8(__ldg(xr + idx), __ldg(G + idx), r);
-      qr[idx] = quant8(u, s);
-      if (nr != nullptr) nr[idx] = u;
+    if (active) {
+      for (int idx = tr + kNqVpt * TPR; idx < nv; idx += TPR) {
+        const uint4 u = norm8(__ldg(xr + idx), __ldg(G + idx), r);
+        qr[idx] = quant8(u, sc);
+        if (nr != nullptr) nr[idx] = u;
+      }
+      if (tr == 0) amax[row] = a;
     }
-    if (tr == 0) amax[row] = a;
   }
 }
 
