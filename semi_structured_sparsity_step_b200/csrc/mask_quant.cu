@@ -332,9 +332,7 @@ __global__ void __launch_bounds__(256) ternary_mask_kernel(const uint4* __restri
                                                            uint8_t* __restrict__ mask_bits) {
   const uint32_t thr = ws->zero_threshold;
   const uint32_t thr2 = thr | (thr << 16);
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_vec;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const uint4 v = __ldg(W + i);
+  auto one = [&](size_t i, const uint4 v) {
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
     // ---- N:M mask from the 15-bit magnitudes
     uint32_t keep = 0u;
@@ -366,7 +364,16 @@ __global__ void __launch_bounds__(256) ternary_mask_kernel(const uint4* __restri
     w_eff[i] = make_uint2(__byte_perm(q16[0], q16[1], 0x6420), __byte_perm(q16[2], q16[3], 0x6420));
     if (w_eff_bf16 != nullptr) w_eff_bf16[i] = make_uint4(qb[0], qb[1], qb[2], qb[3]);
     if (mask_bits != nullptr) mask_bits[i] = static_cast<uint8_t>(keep);
+  };
+  // two vectors per thread and iteration, both loads issued first
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  for (; i + stride < n_vec; i += 2 * stride) {
+    const uint4 v0 = __ldg(W + i), v1 = __ldg(W + i + stride);
+    one(i, v0);
+    one(i + stride, v1);
   }
+  if (i < n_vec) one(i, __ldg(W + i));
 }
 
 // ---------------------------------------------------------------------------
