@@ -76,10 +76,10 @@ sbl_status sbl_set_gemm_variant(int variant);
 
 /* Select the decode GEMV kernel used by sbl_gemv_packed(_group) and
  * sbl_gemv_dense2_group for all later calls in this process: 0 = each warp
- * streams its own rows into registers (the default), 1 = a block-wide TMA
- * tile ring with producer and epilogue warps.  Results are identical (exact
- * int32 sums, the same scaling).  Same threading caveat as
- * sbl_set_gemm_variant. */
+ * streams its own 16-row slices through its own TMA ring in shared memory,
+ * long rows cut into k slices (the default), 1 = one block-wide TMA tile
+ * ring with producer and epilogue warps.  Results are identical (exact int32
+ * sums, the same scaling).  Same threading caveat as sbl_set_gemm_variant. */
 sbl_status sbl_set_gemv_variant(int variant);
 
 /* Synchronise `stream`, then return (and clear) the first error latched by a

@@ -18,8 +18,10 @@
 // group when M = 8, two groups when M = 4.  A chunk has K = 8N/M slots,
 // 2K code bits and 8 index bits (one index byte).
 //
-// Decode GEMV: see gemv_packed_kernel.  One launch can serve a group of
-// independent problems (e.g. the seven projections of a layer).
+// Decode GEMV: gemv_packed_kernel here is the block-wide tile-ring kernel,
+// selected with sbl_set_gemv_variant(1); the default kernel, with a ring per
+// warp, is in gemv_direct.cu.  One launch serves a group of independent
+// problems (e.g. the seven projections of a layer).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
