@@ -10,9 +10,10 @@
 // acc = sum_j W_eff[o, j] * Xq[b, j] exactly in int32, batch <= 16.
 //
 // Work decomposition.  A row block is 16 weight rows of one problem (the
-// rows of one m16n8k32 MMA).  Its k range is cut into slices of at most
-// kSliceStages stages (a stage = 128 chunks = 1024 weights), so slices move
-// about the same number of bytes whatever d_in is.  Row blocks are dealt to
+// rows of one m16n8k32 MMA).  A row of at most kSliceStages stages (a stage =
+// 128 chunks = 1024 weights) is one slice; a longer row is cut into
+// one-stage slices, so a block's slices are small enough to share out evenly
+// over its warps whatever d_in is.  Row blocks are dealt to
 // the persistent blocks (one per SM) round-robin, longest rows first; the
 // block's slices go to its 12 warps round-robin.  Each warp owns a ring of
 // kRing stages in shared memory that its lane 0 fills with 2-D TMA copies
@@ -520,7 +521,10 @@ cudaError_t launch_gemv_direct(const GemvProblemDev* probs, int count, int batch
     d.d_out = q.d_out;
     d.nchunks = q.d_in / 8;
     d.stages = (d.nchunks + kStageChunks - 1) / kStageChunks;
-    d.slices = (d.stages + kSliceStages - 1) / kSliceStages;
+    // rows of up to kSliceStages stages stay whole; longer rows are cut into
+    // one-stage slices, so the warps of a block that owns a long row block
+    // still end up with nearly equal work
+    d.slices = d.stages <= kSliceStages ? 1 : d.stages;
     grp.rb_start[i] = rbs;
     rbs += (q.d_out + 15) / 16;
   }
