@@ -415,8 +415,9 @@ def run_prefill(args):
     (sbl_forward_packed), unpacked once per pass and multiplied by the dense
     int8 kernel (sbl_unpack + sbl_forward), and from an int8 W_eff that is
     already resident (sbl_forward).  Shapes: 512 tokens (1 x 512), 8192
-    (8 x 1024) and 32768 (16 x 2048).  One pass = the seven projections,
-    captured in a CUDA graph; int8 ops = 2 T P (dense-equivalent)."""
+    (8 x 1024) and 32768 (16 x 2048).  One pass = the seven projections;
+    passes are captured in a CUDA graph (16 passes per replay at 512 tokens,
+    2 at 8192, 1 at 32768); int8 ops = 2 T P (dense-equivalent)."""
     import semi_structured_sparsity_step_b200 as sbl
     from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer, act_quant
     torch.cuda.set_device(0)
@@ -465,9 +466,13 @@ def run_prefill(args):
                 for _ in range(2):
                     one_pass(variant)
             stream.synchronize()
-            graph = torch.cuda.CUDAGraph()  # one pass per replay: no host launch cost in the timing
+            # several passes per replay for short passes, so the host's cost of
+            # a replay never shows in the device timing
+            per_graph = 16 if T <= 1024 else (2 if T <= 8192 else 1)
+            graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, stream=stream):
-                one_pass(variant)
+                for _ in range(per_graph):
+                    one_pass(variant)
             for _ in range(args.warmup):
                 graph.replay()
             stream.synchronize()
@@ -481,7 +486,7 @@ def run_prefill(args):
             e1.record(stream)
             stream.synchronize()
             del graph
-            ms = e0.elapsed_time(e1) / reps
+            ms = e0.elapsed_time(e1) / (reps * per_graph)
             tops = 2.0 * T * ls.params / (ms / 1e3) / 1e12
             row[variant] = {"ms_per_pass": ms, "tokens_per_s": T / (ms / 1e3), "int8_tops": tops,
                             "frac_int8_peak": tops / i8_peak}

@@ -42,6 +42,14 @@ constexpr int kThreads = 192;
 
 enum Epi : int { kEpiFwd = 0, kEpiDx = 1, kEpiDw = 2 };
 
+// Programmatic dependent launch: a product may start while the previous
+// kernel of its stream finishes.  The prologue (barriers, tensor memory,
+// descriptor prefetch, the packed-B selector table) touches only kernel
+// parameters and on-chip state; every thread waits for the previous kernel
+// before any global load, TMA copy or store.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 struct GemmArgs {
   int M, N, K;
   int kb_per_split;
@@ -52,6 +60,7 @@ struct GemmArgs {
   const float* gamma;
   int accumulate;  // dW: add into `out`
   int atomic_out;  // split-K: atomically add into `out`
+  int atomic_i32;  // forward split-K: add the int32 partial sums, as exact fp32 integers, into `out`
   uint32_t* err;
 };
 
@@ -101,7 +110,8 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, float* tile, i
   for (int j = 0; j < 32; ++j) {
     float v;
     if constexpr (EPI == kEpiFwd) {
-      v = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scale);
+      v = a.atomic_i32 ? __int2float_rn(static_cast<int>(r[j]))
+                       : __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scale);
     } else if constexpr (EPI == kEpiDx) {
       v = __fmul_rn(scale, __uint_as_float(r[j]));
     } else {
@@ -110,7 +120,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, float* tile, i
     tile[lane * 33 + j] = v;
   }
   if constexpr (EPI == kEpiFwd) {
-    if (a.acc_out != nullptr && row0 + lane < a.M) {
+    if (!a.atomic_i32 && a.acc_out != nullptr && row0 + lane < a.M) {
       int32_t* arow = a.acc_out + static_cast<long long>(row0 + lane) * a.ldo + col0;
 #pragma unroll
       for (int j = 0; j < 32; j += 4)
@@ -130,6 +140,15 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, float* tile, i
       const float* t = tile + rr * 33 + cq;
       float4 v = make_float4(t[0], t[1], t[2], t[3]);
       float* dst = a.out + static_cast<long long>(grow) * a.ldo + gcol;
+      if constexpr (EPI == kEpiFwd) {
+        if (a.atomic_i32) {
+          // one k split's int32 sums as fp32: every partial and total is an
+          // integer below 2^24 in magnitude, so each fp32 addition is exact
+          // and the order of the atomics does not matter
+          atomicAdd(reinterpret_cast<float4*>(dst), v);
+          continue;
+        }
+      }
       if constexpr (EPI == kEpiDw) {
         if (a.atomic_out) {
           atomicAdd(reinterpret_cast<float4*>(dst), v);
@@ -172,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int KB = (args.K + C::BK - 1) / C::BK;
 
+  if (threadIdx.x == 0) pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -194,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -448,6 +469,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
   const int KB = (args.K + C::BK - 1) / C::BK;
   const uint32_t peer_abort = pair::map_to(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
 
+  if (threadIdx.x == 0) pdl_launch_dependents();
   if constexpr (KP > 0) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) {
       uint32_t s0, s1;
@@ -481,6 +503,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
   pair::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated, tables built
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
 
   auto give_up = [&]() {
     *abort_flag = 1;
@@ -745,6 +768,23 @@ bool make_tmap_u8(CUtensorMap* m, const void* base, unsigned long long inner, un
 
 namespace {
 
+// Launch with programmatic stream serialization (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int threads, int smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 template <bool kI8, bool kAMN, bool kBMN, int BN, int STAGES, int EPI>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int splits, int num_sms,
                 cudaStream_t stream) {
@@ -759,8 +799,7 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
   sc.total = sc.Mt * sc.Nt * splits;
   sc.GM = 1;
   const int grid = sc.total < num_sms ? sc.total : num_sms;
-  kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(ta, tb, a, sc);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, kThreads, C::SMEM_BYTES, stream, ta, tb, a, sc);
 }
 
 // Strip height (m blocks) that minimises the estimated DRAM bytes of the
@@ -804,8 +843,7 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArg
   int pairs = num_sms / 2;
   if (pairs > sc.total) pairs = sc.total;
   sc.GM = pick_strip(sc.Mt, sc.Nt, pairs, a_bytes, b_bytes);
-  kern<<<2 * pairs, C::THREADS, C::SMEM_BYTES, stream>>>(ta, tb, a, sc, pb);
-  return cudaGetLastError();
+  return launch_pdl(kern, 2 * pairs, C::THREADS, C::SMEM_BYTES, stream, ta, tb, a, sc, pb);
 }
 
 constexpr int kBN = 256;
@@ -822,6 +860,29 @@ int g_gemm_variant = 0;
 
 namespace {
 
+}  // namespace
+
+namespace {
+// Forward with split K: the GEMM has added the exact integer sums into Y as
+// fp32 values (|acc| <= 128 d_in < 2^24); turn them into y = fp32(acc) *
+// fp32(gamma * fp32(amax_t / 127)) in place, with the same operations as the
+// GEMM epilogue, and copy the sums to `acc` when it is given.  d_out % 8 ==
+// 0, so a 16-byte vector never straddles two rows.
+__global__ void __launch_bounds__(256) fwd_split_finalize_kernel(float4* __restrict__ Y, int4* __restrict__ acc,
+                                                                 const float* __restrict__ amax,
+                                                                 const float* __restrict__ gamma, int d_out,
+                                                                 size_t n4) {
+  const float gm = *gamma;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>((4 * i) / static_cast<size_t>(d_out));
+    const float sc = __fmul_rn(gm, __fdiv_rn(amax[row], 127.0f));
+    const float4 f = Y[i];  // exact integers
+    if (acc != nullptr)
+      acc[i] = make_int4(__float2int_rn(f.x), __float2int_rn(f.y), __float2int_rn(f.z), __float2int_rn(f.w));
+    Y[i] = make_float4(__fmul_rn(f.x, sc), __fmul_rn(f.y, sc), __fmul_rn(f.z, sc), __fmul_rn(f.w, sc));
+  }
+}
 }  // namespace
 
 cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
@@ -849,10 +910,41 @@ cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_
   a.amax = amax;
   a.gamma = gamma;
   a.err = err;
-  if (use_pair)
+  if (use_pair) {
+    // Few output tiles (a short token batch): split K so every CTA pair has
+    // work.  The splits add their exact integer sums into Y, which a second
+    // pass scales in place (bit-identical to the unsplit product).
+    const int KB = (d_in + 127) / 128;
+    const int tiles = ((T + 255) / 256) * ((d_out + 255) / 256);
+    const int pairs = num_sms / 2;
+    int splits = 1;
+    if (tiles < pairs && d_in < (1 << 17)) {  // 128 * d_in < 2^24: exact fp32 partial sums
+      splits = pairs / tiles;
+      if (splits > KB / 4) splits = KB / 4;  // at least four K blocks per split
+      if (splits < 1) splits = 1;
+    }
+    if (splits > 1) {
+      a.kb_per_split = (KB + splits - 1) / splits;
+      splits = (KB + a.kb_per_split - 1) / a.kb_per_split;
+      a.atomic_i32 = 1;
+      const size_t n = static_cast<size_t>(T) * d_out;
+      cudaError_t e = cudaMemsetAsync(Y, 0, sizeof(float) * n, stream);
+      if (e != cudaSuccess) return e;
+      e = run_pair<true, false, false, kPairStages, kEpiFwd>(ta, tb, a, splits, num_sms, stream,
+                                                             static_cast<double>(T) * d_in,
+                                                             static_cast<double>(d_out) * d_in);
+      if (e != cudaSuccess) return e;
+      const size_t n4 = n / 4;
+      size_t blocks = (n4 + 255) / 256;
+      if (blocks > static_cast<size_t>(num_sms) * 8) blocks = static_cast<size_t>(num_sms) * 8;
+      fwd_split_finalize_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+          reinterpret_cast<float4*>(Y), reinterpret_cast<int4*>(acc), amax, gamma, d_out, n4);
+      return cudaGetLastError();
+    }
     return run_pair<true, false, false, kPairStages, kEpiFwd>(ta, tb, a, 1, num_sms, stream,
                                                              static_cast<double>(T) * d_in,
                                                              static_cast<double>(d_out) * d_in);
+  }
   return run<true, false, false, kBN, kStages, kEpiFwd>(ta, tb, a, 1, num_sms, stream);
 }
 
