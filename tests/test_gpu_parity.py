@@ -284,6 +284,32 @@ def test_gemv_group_matches_single_calls(lib, gemv_variant, batch):
         assert np.array_equal(Y.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("T,d_out,d_in", [(64, 512, 11008), (300, 264, 4368), (512, 2048, 2048), (17, 8, 16384)])
+@pytest.mark.parametrize("variant", [0, 1])
+def test_forward_split_k_exact(lib, T, d_out, d_in, variant):
+    """Short token batches with long rows: the CTA-pair forward splits K
+    (fewer output tiles than CTA pairs) and its splits add exact integer
+    sums that a finalize pass scales; y and the int32 accumulators must equal
+    the oracle's exactly, as for the unsplit one-CTA kernel."""
+    w = synth.trimodal_weight(d_out, d_in, seed=46, tensor_id=d_in)
+    x = synth.activations(T, d_in, seed=46, tensor_id=100 + T, outlier_frac=0.01)
+    weff, gamma, _ = oracle.effective_weight(synth.bits(w), 6, 8)
+    xq, amax = oracle.act_quant(synth.bits(x))
+    Y = torch.full((T, d_out), float("nan"), dtype=torch.float32, device="cuda")
+    acc = torch.empty(T, d_out, dtype=torch.int32, device="cuda")
+    g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+    lib.sbl_set_gemm_variant(variant)
+    try:
+        lib.sbl_forward(torch.from_numpy(xq).cuda(), torch.from_numpy(amax).cuda(), torch.from_numpy(weff).cuda(),
+                        g, T, d_in, d_out, Y, acc)
+        lib.sbl_check()
+    finally:
+        lib.sbl_set_gemm_variant(0)
+    racc = oracle.forward_acc(xq, weff)
+    assert np.array_equal(acc.cpu().numpy(), racc)
+    assert np.array_equal(Y.cpu().numpy(), oracle.forward_out(racc, gamma, amax))
+
+
 @pytest.mark.parametrize("T,d_out,d_in,N,M", [
     (64, 256, 256, 6, 8), (300, 264, 2064, 6, 8), (129, 520, 1040, 2, 4), (257, 136, 400, 4, 8),
     (100, 392, 2048, 8, 8), (33, 8, 4864, 1, 8), (77, 128, 272, 3, 4),
