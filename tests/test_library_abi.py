@@ -25,7 +25,7 @@ def _declared():
     return sorted(set(re.findall(r"\b(sbl_[a-z0-9_]+)\s*\(", src)))
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_core_entry_points():
     names = _declared()
     for n in ["sbl_mask_quant", "sbl_act_quant", "sbl_forward", "sbl_backward", "sbl_pack", "sbl_gemv_packed",
               "sbl_check", "sbl_status_string", "sbl_packed_bytes"]:
