@@ -411,10 +411,11 @@ def _decode_pass_ms(sbl, stream, groups, batch, variant, args):
 def run_prefill(args):
     """Prefill forward on the packed 6:8 format of the 3B layer set: per
     projection, int8 activations (absmax-quantised N(0, 1)) times the packed
-    weight, three ways: expanded in shared memory for every token tile
+    weight: expanded in shared memory for every token tile
     (sbl_forward_packed), unpacked once per pass and multiplied by the dense
-    int8 kernel (sbl_unpack + sbl_forward), and from an int8 W_eff that is
-    already resident (sbl_forward).  Shapes: 512 tokens (1 x 512), 8192
+    int8 kernel (sbl_unpack + sbl_forward_group), and from an int8 W_eff that
+    is already resident (sbl_forward per projection, and sbl_forward_group,
+    which runs short batches in one launch).  Shapes: 512 tokens (1 x 512), 8192
     (8 x 1024) and 32768 (16 x 2048).  One pass = the seven projections;
     passes are captured in a CUDA graph (16 passes per replay at 512 tokens,
     2 at 8192, 1 at 32768); int8 ops = 2 T P (dense-equivalent)."""
@@ -454,14 +455,17 @@ def run_prefill(args):
                 xq, am = xs[p.input_name]
                 if variant == "packed":      # weight decoded in shared memory for every token tile
                     sbl.sbl_forward_packed(xq, am, pk, L.gamma, T, p.d_in, p.d_out, N_KEEP, M_GROUP, y, None, stream)
-                elif variant == "unpack_int8":  # decoded once per pass, then the dense int8 product
+                elif variant == "unpack_int8":  # decoded once per pass, then the dense int8 products
                     sbl.sbl_unpack(pk, p.d_out, p.d_in, N_KEEP, M_GROUP, wk, stream)
-                    sbl.sbl_forward(xq, am, wk, L.gamma, T, p.d_in, p.d_out, y, None, stream)
-                else:                        # int8 W_eff already resident (training layout)
+                elif variant == "int8_weff":  # int8 W_eff already resident (training layout)
                     sbl.sbl_forward(xq, am, L.W_eff, L.gamma, T, p.d_in, p.d_out, y, None, stream)
+            if variant in ("unpack_int8", "int8_weff_grouped"):  # the seven products through sbl_forward_group
+                weights = unpacked if variant == "unpack_int8" else [L.W_eff for (_, L, _) in layers]
+                sbl.sbl_forward_group([(xs[p.input_name][0], xs[p.input_name][1], w, L.gamma, T, p.d_in, p.d_out,
+                                        y, None) for (p, L, _), y, w in zip(layers, ys, weights)], stream)
 
         row = {}
-        for variant in ("packed", "unpack_int8", "int8_weff"):
+        for variant in ("packed", "unpack_int8", "int8_weff", "int8_weff_grouped"):
             with torch.cuda.stream(stream):
                 for _ in range(2):
                     one_pass(variant)

@@ -258,6 +258,26 @@ sbl_status sbl_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff,
                        const float* gamma, int T, int d_in, int d_out, float* Y,
                        int32_t* acc, void* stream);
 
+/* Several forward products (e.g. the seven projections of a layer):
+ * problem i is exactly sbl_forward on its own buffers.  While the products
+ * together have at most four 256 x 256 output tiles per pair of SMs (short
+ * token batches, such as a prefill of a few hundred tokens) they run in one
+ * launch, which pays the fixed start-up cost once; larger ones run one launch
+ * each.  Same citation as sbl_forward.
+ *   problems  HOST array of `count` descriptors (read before the call
+ *             returns; the pointers inside are device pointers); each is
+ *             validated as sbl_forward validates its arguments. */
+typedef struct {
+  const int8_t* Xq;     /* [T, d_in] int8                          */
+  const float* amax;    /* [T] float                               */
+  const int8_t* W_eff;  /* [d_out, d_in] int8                      */
+  const float* gamma;   /* 1 float (device)                        */
+  int T, d_in, d_out;
+  float* Y;             /* [T, d_out] float out                    */
+  int32_t* acc;         /* optional [T, d_out] int32 out (NULL)    */
+} sbl_forward_problem;
+sbl_status sbl_forward_group(const sbl_forward_problem* problems, int count, void* stream);
+
 /* Forward product with the weight read from the packed format (prefill on a
  * deployed model): the same result as sbl_forward on the unpacked W_eff, bit
  * for bit.  [summary] Algorithm 1 step (6); [article] 7.1 (cached sparse

@@ -18,6 +18,12 @@ _c_int = ctypes.c_int
 _c_size = ctypes.c_size_t
 _vp = ctypes.c_void_p
 
+class ForwardProblem(ctypes.Structure):
+    """sbl_forward_problem: one product of a grouped forward (device pointers)."""
+    _fields_ = [("Xq", _vp), ("amax", _vp), ("W_eff", _vp), ("gamma", _vp), ("T", _c_int), ("d_in", _c_int),
+                ("d_out", _c_int), ("Y", _vp), ("acc", _vp)]
+
+
 class GemvProblem(ctypes.Structure):
     """sbl_gemv_problem: one decode GEMV of a group (device pointers)."""
     _fields_ = [("packed", _vp), ("Xq", _vp), ("amax", _vp), ("gamma", _vp), ("Y", _vp),
@@ -47,6 +53,7 @@ SIGNATURES = {
     "sbl_rmsnorm_act_quant": (_c_int, [_vp, _vp, ctypes.c_float, _c_int, _c_int, _vp, _vp, _vp, _vp]),
     "sbl_forward": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "sbl_forward_packed": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
+    "sbl_forward_group": (_c_int, [_vp, _c_int, _vp]),
     "sbl_compress24_bytes": (_c_size, [_c_int, _c_int]),
     "sbl_compress24": (_c_int, [_vp, _c_int, _c_int, _vp, _c_size, _vp]),
     "sbl_forward_sparse24": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
@@ -198,6 +205,14 @@ def sbl_rmsnorm_act_quant(X, g, eps, T, d_in, Xn, Xq, amax, stream=None) -> None
 def sbl_forward(Xq, amax, W_eff, gamma, T, d_in, d_out, Y, acc=None, stream=None) -> None:
     _call("sbl_forward", _ptr(Xq), _ptr(amax), _ptr(W_eff), _ptr(gamma), T, d_in, d_out, _ptr(Y), _ptr(acc),
           _stream(stream))
+
+
+def sbl_forward_group(problems, stream=None) -> None:
+    """problems: list of (Xq, amax, W_eff, gamma, T, d_in, d_out, Y, acc_or_None)."""
+    arr = (ForwardProblem * max(1, len(problems)))()
+    for i, (xq, am, w, g, T, d_in, d_out, y, acc) in enumerate(problems):
+        arr[i] = ForwardProblem(_ptr(xq), _ptr(am), _ptr(w), _ptr(g), T, d_in, d_out, _ptr(y), _ptr(acc))
+    _call("sbl_forward_group", ctypes.cast(arr, _vp), len(problems), _stream(stream))
 
 
 def sbl_forward_packed(Xq, amax, packed, gamma, T, d_in, d_out, N, M, Y, acc=None, stream=None) -> None:

@@ -443,10 +443,32 @@ __device__ __forceinline__ void expand_packed_half(const PackedHalf<KP>& ph, int
   }
 }
 
-template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI, int KP = 0>
+// Several independent products in one launch (the projections of a layer):
+// per problem its two tensor maps, arguments and tile schedule; work items
+// are numbered problem after problem (the host orders problems heaviest
+// first), and every role of the kernel finds an item's problem the same way.
+// G = 1 is the single product.
+template <int G>
+struct alignas(64) PairGroup {
+  CUtensorMap tmA[G];
+  CUtensorMap tmB[G];
+  GemmArgs args[G];
+  Sched sched[G];
+  int item_start[G + 1];
+  int count, total;
+  __device__ __forceinline__ void locate(int w, int& p, int& mb, int& nb, int& sp) const {
+    p = 0;
+    if constexpr (G > 1) {
+      while (p + 1 < count && w >= item_start[p + 1]) ++p;
+    }
+    sched[p].item(w - item_start[p], mb, nb, sp);
+  }
+};
+
+template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI, int KP = 0, int G = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThreads, 1)
-    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmArgs args, const Sched sched, const PackedB pb) {
+    tc_gemm_pair_kernel(const __grid_constant__ PairGroup<G> grp, const PackedB pb) {
+  const GemmArgs& args = grp.args[0];  // fields shared by the group (err) and the single product
   using C = Cfg2<kI8, kAMN, kBMN, STAGES, KP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -466,7 +488,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
   const bool leader = rank == 0;
   const int pair_id = blockIdx.x >> 1;
   const int n_pairs = gridDim.x >> 1;
-  const int KB = (args.K + C::BK - 1) / C::BK;
   const uint32_t peer_abort = pair::map_to(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
 
   if (threadIdx.x == 0) pdl_launch_dependents();
@@ -492,8 +513,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
     }
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmA);
-    if constexpr (KP == 0) tma_prefetch_desc(&tmB);
+    for (int i = 0; i < grp.count; ++i) {
+      tma_prefetch_desc(&grp.tmA[i]);
+      if constexpr (KP == 0) tma_prefetch_desc(&grp.tmB[i]);
+    }
   }
   if (warp == 1) {
     pair::tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -514,11 +537,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
     if (lane == 0) {
       int it = 0;
       bool ok = true;
-      for (int w = pair_id; w < sched.total && ok; w += n_pairs) {
-        int mb, nb, sp;
-        sched.item(w, mb, nb, sp);
-        const int kb0 = sp * args.kb_per_split;
-        const int kb1 = min(KB, kb0 + args.kb_per_split);
+      for (int w = pair_id; w < grp.total && ok; w += n_pairs) {
+        int pi, mb, nb, sp;
+        grp.locate(w, pi, mb, nb, sp);
+        const GemmArgs& A = grp.args[pi];
+        const CUtensorMap* tmA = &grp.tmA[pi];
+        const CUtensorMap* tmB = &grp.tmB[pi];
+        const int KB = (A.K + C::BK - 1) / C::BK;
+        const int kb0 = sp * A.kb_per_split;
+        const int kb1 = min(KB, kb0 + A.kb_per_split);
         const int m0 = mb * 256 + 128 * static_cast<int>(rank);
         const int n0 = nb * C::BN + 128 * static_cast<int>(rank);
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -535,17 +562,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
           uint8_t* sb = sa + C::A_BYTES;
           const int kc = kb * C::BK;
           if constexpr (!kAMN) {
-            pair::tma_load_2d(sa, &tmA, fbar, kc, m0);
+            pair::tma_load_2d(sa, tmA, fbar, kc, m0);
           } else {
-            pair::tma_load_2d(sa, &tmA, fbar, m0, kc);
-            pair::tma_load_2d(sa + C::BK * 128, &tmA, fbar, m0 + 64, kc);
+            pair::tma_load_2d(sa, tmA, fbar, m0, kc);
+            pair::tma_load_2d(sa + C::BK * 128, tmA, fbar, m0 + 64, kc);
           }
           if constexpr (KP == 0) {
             if constexpr (!kBMN) {
-              pair::tma_load_2d(sb, &tmB, fbar, kc, n0);
+              pair::tma_load_2d(sb, tmB, fbar, kc, n0);
             } else {
-              pair::tma_load_2d(sb, &tmB, fbar, n0, kc);
-              pair::tma_load_2d(sb + C::BK * 128, &tmB, fbar, n0 + 64, kc);
+              pair::tma_load_2d(sb, tmB, fbar, n0, kc);
+              pair::tma_load_2d(sb + C::BK * 128, tmB, fbar, n0 + 64, kc);
             }
           }
           ++it;
@@ -560,11 +587,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
     if (lane == 0 && leader) {
       int it = 0, t = 0;
       bool ok = true;
-      for (int w = pair_id; w < sched.total && ok; w += n_pairs, ++t) {
-        int mb, nb, sp;
-        sched.item(w, mb, nb, sp);
-        const int kb0 = sp * args.kb_per_split;
-        const int kb1 = min(KB, kb0 + args.kb_per_split);
+      for (int w = pair_id; w < grp.total && ok; w += n_pairs, ++t) {
+        int pi, mb, nb, sp;
+        grp.locate(w, pi, mb, nb, sp);
+        const GemmArgs& A = grp.args[pi];
+        const int KB = (A.K + C::BK - 1) / C::BK;
+        const int kb0 = sp * A.kb_per_split;
+        const int kb1 = min(KB, kb0 + A.kb_per_split);
         const int b = t & 1;
         if (!mbar_wait(&tempty[b], (static_cast<uint32_t>(t >> 1) & 1u) ^ 1u, abort_flag, args.err)) {
           give_up();
@@ -605,6 +634,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
       const int dt = (warp - 6) * 32 + lane;
       const int r = dt & 127, hf = dt >> 7;
       const int nchunks = args.K / 8;
+      const int KB = (args.K + C::BK - 1) / C::BK;
+      const Sched& sched = grp.sched[0];
       // Walk the same (item, k block) sequence as the TMA producer; the
       // packed words of the next k block are loaded (from L2) into registers
       // before waiting for the current stage, hiding the load latency.
@@ -616,16 +647,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
         kb1 = min(KB, kb + args.kb_per_split);
         row = nb * C::BN + 128 * static_cast<int>(rank) + r;
       };
-      if (w < sched.total) start_item(w);
+      if (w < grp.total) start_item(w);
       PackedHalf<KP> cur, nxt;
-      if (w < sched.total) load_packed_half<KP>(cur, pb, row, kb, hf, nchunks);
+      if (w < grp.total) load_packed_half<KP>(cur, pb, row, kb, hf, nchunks);
       int it = 0;
-      while (w < sched.total) {
+      while (w < grp.total) {
         // position of the next k block in the sequence
         int nw = w, nkb = kb + 1, nkb1 = kb1, nrow = row;
         if (nkb >= kb1) {
           nw = w + n_pairs;
-          if (nw < sched.total) {
+          if (nw < grp.total) {
             int mb, nb, sp;
             sched.item(nw, mb, nb, sp);
             nkb = sp * args.kb_per_split;
@@ -633,7 +664,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
             nrow = nb * C::BN + 128 * static_cast<int>(rank) + r;
           }
         }
-        if (nw < sched.total) load_packed_half<KP>(nxt, pb, nrow, nkb, hf, nchunks);
+        if (nw < grp.total) load_packed_half<KP>(nxt, pb, nrow, nkb, hf, nchunks);
         const int s = it % STAGES;
         const uint32_t round = static_cast<uint32_t>(it / STAGES);
         const bool waited = mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, args.err);
@@ -662,9 +693,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
     const int q = warp & 3;
     float* tile = epi_tiles + q * C::EPI_WARP_FLOATS;
     int t = 0;
-    for (int w = pair_id; w < sched.total; w += n_pairs, ++t) {
-      int mb, nb, sp;
-      sched.item(w, mb, nb, sp);
+    for (int w = pair_id; w < grp.total; w += n_pairs, ++t) {
+      int pi, mb, nb, sp;
+      grp.locate(w, pi, mb, nb, sp);
+      const GemmArgs& A = grp.args[pi];
       const int b = t & 1;
       if (!mbar_wait(&tfull[b], static_cast<uint32_t>(t >> 1) & 1u, abort_flag, args.err)) {
         give_up();
@@ -676,19 +708,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP > 0 ? 448 : kThre
       const int row = row0 + lane;
       float scale = 0.0f;
       if constexpr (EPI == kEpiFwd) {
-        if (row < args.M) scale = __fmul_rn(*args.gamma, __fdiv_rn(args.amax[row], 127.0f));
+        if (row < A.M) scale = __fmul_rn(*A.gamma, __fdiv_rn(A.amax[row], 127.0f));
       } else if constexpr (EPI == kEpiDx) {
-        scale = *args.gamma;
+        scale = *A.gamma;
       }
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b * C::BN);
 #pragma unroll 1
       for (int c = 0; c < C::BN / 32; ++c) {
         const int col0 = nb * C::BN + 32 * c;
-        if (col0 >= args.N) break;  // warp-uniform
+        if (col0 >= A.N) break;  // warp-uniform
         uint32_t r[32];
         tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(32 * c), r);
         tmem_ld_wait();
-        epilogue_chunk<EPI>(args, tile, row0, col0, lane, r, scale);
+        epilogue_chunk<EPI>(A, tile, row0, col0, lane, r, scale);
       }
       tc_fence_before();
       __syncwarp();
@@ -832,7 +864,7 @@ template <bool kI8, bool kAMN, bool kBMN, int STAGES, int EPI, int KP = 0>
 cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int splits, int num_sms,
                      cudaStream_t stream, double a_bytes, double b_bytes, const PackedB& pb = PackedB{}) {
   using C = Cfg2<kI8, kAMN, kBMN, STAGES, KP>;
-  auto kern = tc_gemm_pair_kernel<kI8, kAMN, kBMN, STAGES, EPI, KP>;
+  auto kern = tc_gemm_pair_kernel<kI8, kAMN, kBMN, STAGES, EPI, KP, 1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   Sched sc;
@@ -843,8 +875,19 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArg
   int pairs = num_sms / 2;
   if (pairs > sc.total) pairs = sc.total;
   sc.GM = pick_strip(sc.Mt, sc.Nt, pairs, a_bytes, b_bytes);
-  return launch_pdl(kern, 2 * pairs, C::THREADS, C::SMEM_BYTES, stream, ta, tb, a, sc, pb);
+  PairGroup<1> grp{};
+  grp.tmA[0] = ta;
+  grp.tmB[0] = tb;
+  grp.args[0] = a;
+  grp.sched[0] = sc;
+  grp.item_start[0] = 0;
+  grp.item_start[1] = sc.total;
+  grp.count = 1;
+  grp.total = sc.total;
+  return launch_pdl(kern, 2 * pairs, C::THREADS, C::SMEM_BYTES, stream, grp, pb);
 }
+
+constexpr int kFwdGroup = 8;  // products of one grouped forward launch at most
 
 constexpr int kBN = 256;
 constexpr int kStages = 4;
@@ -946,6 +989,92 @@ cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_
                                                              static_cast<double>(d_out) * d_in);
   }
   return run<true, false, false, kBN, kStages, kEpiFwd>(ta, tb, a, 1, num_sms, stream);
+}
+
+cudaError_t launch_forward_group(const FwdProblemDev* probs, int count, cudaStream_t stream, int num_sms,
+                                 uint32_t* err) {
+  // One launch pays the start-up cost once, which is what short token batches
+  // need; products that are large together run one by one instead, where each
+  // launch keeps its own operands' reuse in L2 (measured: grouping the seven
+  // 3B projections halves the pass at 512 tokens and slows it at 32768).
+  long long tiles = 0;
+  for (int i = 0; i < count; ++i)
+    if (probs[i].T > 0 && probs[i].d_out > 0)
+      tiles += static_cast<long long>((probs[i].T + 255) / 256) * ((probs[i].d_out + 255) / 256);
+  if (g_gemm_variant != 0 || tiles > 4LL * (num_sms / 2)) {  // one launch per product
+    for (int i = 0; i < count; ++i) {
+      const FwdProblemDev& q = probs[i];
+      const cudaError_t e = launch_forward(q.Xq, q.amax, q.W_eff, q.gamma, q.T, q.d_in, q.d_out, q.Y, q.acc, stream,
+                                           num_sms, err);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  using C = Cfg2<true, false, false, kPairStages, 0>;
+  for (int c0 = 0; c0 < count; c0 += kFwdGroup) {
+    const int cnt = (count - c0) < kFwdGroup ? (count - c0) : kFwdGroup;
+    // longest K first: those items take longest and should start first
+    int order[kFwdGroup];
+    int n = 0;
+    for (int i = 0; i < cnt; ++i) {
+      const FwdProblemDev& q = probs[c0 + i];
+      if (q.T == 0 || q.d_out == 0) continue;
+      if (q.d_in == 0) {  // an empty product: zeros
+        cudaError_t e = cudaMemsetAsync(q.Y, 0, sizeof(float) * static_cast<size_t>(q.T) * q.d_out, stream);
+        if (e == cudaSuccess && q.acc != nullptr)
+          e = cudaMemsetAsync(q.acc, 0, sizeof(int32_t) * static_cast<size_t>(q.T) * q.d_out, stream);
+        if (e != cudaSuccess) return e;
+        continue;
+      }
+      order[n++] = c0 + i;
+    }
+    for (int i = 1; i < n; ++i)
+      for (int k = i; k > 0 && probs[order[k]].d_in > probs[order[k - 1]].d_in; --k) {
+        const int tmp = order[k];
+        order[k] = order[k - 1];
+        order[k - 1] = tmp;
+      }
+    if (n == 0) continue;
+    PairGroup<kFwdGroup> grp{};
+    int total = 0;
+    for (int i = 0; i < n; ++i) {
+      const FwdProblemDev& q = probs[order[i]];
+      if (!make_tmap(&grp.tmA[i], q.Xq, false, q.d_in, q.T, q.d_in, 128, BM)) return cudaErrorInvalidValue;
+      if (!make_tmap(&grp.tmB[i], q.W_eff, false, q.d_in, q.d_out, q.d_in, 128, 128)) return cudaErrorInvalidValue;
+      GemmArgs& a = grp.args[i];
+      a = GemmArgs{};
+      a.M = q.T;
+      a.N = q.d_out;
+      a.K = q.d_in;
+      a.kb_per_split = (q.d_in + 127) / 128;
+      a.out = q.Y;
+      a.ldo = q.d_out;
+      a.acc_out = q.acc;
+      a.amax = q.amax;
+      a.gamma = q.gamma;
+      a.err = err;
+      Sched& sc = grp.sched[i];
+      sc.Mt = (q.T + 255) / 256;
+      sc.Nt = (q.d_out + C::BN - 1) / C::BN;
+      sc.splits = 1;
+      sc.total = sc.Mt * sc.Nt;
+      sc.GM = pick_strip(sc.Mt, sc.Nt, num_sms / 2, static_cast<double>(q.T) * q.d_in,
+                         static_cast<double>(q.d_out) * q.d_in);
+      grp.item_start[i] = total;
+      total += sc.total;
+    }
+    grp.item_start[n] = total;
+    grp.count = n;
+    grp.total = total;
+    int pairs = num_sms / 2;
+    if (pairs > total) pairs = total;
+    auto kern = tc_gemm_pair_kernel<true, false, false, kPairStages, kEpiFwd, 0, kFwdGroup>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(kern, 2 * pairs, C::THREADS, C::SMEM_BYTES, stream, grp, PackedB{});
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_backward(const void* dY, const void* X, const void* W_eff_bf16, const float* gamma, int T,

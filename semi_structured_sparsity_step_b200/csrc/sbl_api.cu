@@ -268,6 +268,32 @@ sbl_status sbl_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff,
                                   d->num_sms, d->err));
 }
 
+sbl_status sbl_forward_group(const sbl_forward_problem* problems, int count, void* stream) {
+  if (count < 0 || (count > 0 && problems == nullptr)) return SBL_ERR_INVALID_ARG;
+  if (count == 0) return SBL_OK;
+  std::vector<FwdProblemDev> dev;
+  dev.reserve(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    const sbl_forward_problem& q = problems[i];
+    sbl_status st = check_dims(q.d_in, q.d_out);
+    if (st != SBL_OK) return st;
+    if (q.T < 0) return SBL_ERR_SHAPE;
+    if (q.T == 0 || q.d_out == 0) continue;
+    if (q.Xq == nullptr || q.amax == nullptr || q.W_eff == nullptr || q.gamma == nullptr || q.Y == nullptr)
+      return SBL_ERR_INVALID_ARG;
+    if (!aligned16(q.Xq) || !aligned16(q.amax) || !aligned16(q.W_eff) || !aligned16(q.Y) || !aligned16(q.acc) ||
+        (reinterpret_cast<uintptr_t>(q.gamma) & 3u) != 0)
+      return SBL_ERR_ALIGN;
+    dev.push_back(FwdProblemDev{q.Xq, q.amax, q.W_eff, q.gamma, q.T, q.d_in, q.d_out, q.Y, q.acc});
+  }
+  if (dev.empty()) return SBL_OK;
+  DeviceInfo* d = nullptr;
+  const sbl_status st = current_device(&d);
+  if (st != SBL_OK) return st;
+  return from_cuda(launch_forward_group(dev.data(), static_cast<int>(dev.size()), static_cast<cudaStream_t>(stream),
+                                        d->num_sms, d->err));
+}
+
 sbl_status sbl_forward_packed(const int8_t* Xq, const float* amax, const uint8_t* packed, const float* gamma,
                               int T, int d_in, int d_out, int N, int M, float* Y, int32_t* acc, void* stream) {
   sbl_status st = check_nm(N, M);

@@ -61,6 +61,18 @@ extern int g_gemm_variant;
 cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
                            int d_in, int d_out, float* Y, int32_t* acc, cudaStream_t stream, int num_sms,
                            uint32_t* err);
+// One problem of a grouped forward (device pointers).
+struct FwdProblemDev {
+  const int8_t* Xq;
+  const float* amax;
+  const int8_t* W_eff;
+  const float* gamma;
+  int T, d_in, d_out;
+  float* Y;
+  int32_t* acc;
+};
+cudaError_t launch_forward_group(const FwdProblemDev* probs, int count, cudaStream_t stream, int num_sms,
+                                 uint32_t* err);
 cudaError_t launch_forward_packed(const int8_t* Xq, const float* amax, const uint8_t* packed, const float* gamma,
                                   int T, int d_in, int d_out, int N, int M, float* Y, int32_t* acc,
                                   cudaStream_t stream, int num_sms, uint32_t* err);

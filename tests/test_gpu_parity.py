@@ -284,6 +284,44 @@ def test_gemv_group_matches_single_calls(lib, gemv_variant, batch):
         assert np.array_equal(Y.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("variant", [0, 1])
+def test_forward_group_matches_single_calls(lib, variant):
+    """One grouped launch over products of different shapes (ragged tokens,
+    rows and d_in; a long-K product; an empty product and a zero-token one)
+    gives each product's exact int32 sums and outputs."""
+    T = 300
+    shapes = [(264, 2048), (8, 896), (520, 11008), (136, 4368), (2048, 256), (40, 0), (16, 64)]
+    toks = [T, T, T, 129, T, T, 0]
+    probs, refs = [], []
+    for i, ((d_out, d_in), t) in enumerate(zip(shapes, toks)):
+        w = synth.trimodal_weight(d_out, max(d_in, 16), seed=47, tensor_id=i)[:, :d_in].contiguous()
+        x = synth.activations(t, max(d_in, 16), seed=47, tensor_id=100 + i)[:, :d_in].contiguous()
+        weff, gamma, _ = oracle.effective_weight(synth.bits(w), 6, 8) if d_in else (
+            np.zeros((d_out, 0), np.int8), np.float32(0.0), None)
+        xq, amax = oracle.act_quant(synth.bits(x)) if d_in else (np.zeros((t, 0), np.int8), np.ones(t, np.float32))
+        Y = torch.full((t, d_out), float("nan"), dtype=torch.float32, device="cuda")
+        acc = torch.full((t, d_out), 7, dtype=torch.int32, device="cuda")
+        g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+        xq_d = torch.from_numpy(xq).cuda() if d_in else torch.empty((max(t, 1), 16), dtype=torch.int8, device="cuda")
+        w_d = torch.from_numpy(weff).cuda() if d_in else torch.empty((d_out, 16), dtype=torch.int8, device="cuda")
+        probs.append((xq_d, torch.from_numpy(amax).cuda() if t else torch.ones(1, device="cuda"), w_d, g, t, d_in,
+                      d_out, Y, acc))
+        racc = oracle.forward_acc(xq, weff) if d_in else np.zeros((t, d_out), np.int32)
+        refs.append((racc, oracle.forward_out(racc, gamma, amax) if t else np.zeros((0, d_out), np.float32)))
+    lib.sbl_set_gemm_variant(variant)
+    try:
+        lib.sbl_forward_group(probs)
+        lib.sbl_check()
+    finally:
+        lib.sbl_set_gemm_variant(0)
+    for (_, _, _, _, t, d_in, d_out, Y, acc), (racc, ry) in zip(probs, refs):
+        assert np.array_equal(acc.cpu().numpy(), racc), (t, d_in, d_out)
+        if d_in:
+            assert np.array_equal(Y.cpu().numpy(), ry), (t, d_in, d_out)
+        else:
+            assert not Y.cpu().numpy().any()
+
+
 @pytest.mark.parametrize("T,d_out,d_in", [(64, 512, 11008), (300, 264, 4368), (512, 2048, 2048), (17, 8, 16384)])
 @pytest.mark.parametrize("variant", [0, 1])
 def test_forward_split_k_exact(lib, T, d_out, d_in, variant):
