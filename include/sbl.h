@@ -353,14 +353,20 @@ sbl_status sbl_backward(const void* dY, const void* X, const void* W_eff_bf16,
  * [article] 7.1 (pre-compute and cache the sparse format for inference);
  * [summary] 核心方法 (masking after quantisation makes the deployed ternary
  * weights N:M-structured).
- * Layout, per weight row, two planes each padded to a multiple of 16 bytes:
- *   codes plane: for every group of M, the N slot codes in ascending position
- *     order, 2 bits each (00 = 0, 01 = +1, 11 = -1), as a little-endian bit
- *     stream (code i of group g at bit 2*(g*N + i));
+ * Layout, per weight row, two planes each padded with zero bytes to a
+ * multiple of 16 bytes.  A chunk is 8 consecutive positions; it holds
+ * K = 8N/M slots s_0 < ... < s_(K-1) (its groups' slots in position order),
+ * and H = ceil(K/2).
+ *   codes plane: one 2K-bit field per chunk, little-endian, chunk c at bit
+ *     2K*c.  Inside a field the code of s_q (q < H) sits at bits 4q..4q+1
+ *     and the code of s_(H+q) at bits 4q+2..4q+3; codes +1 = 00, -1 = 01,
+ *     0 = 10.
  *   index plane: the M-bit slot mask of every group (bit p = position p is a
- *     slot), little-endian bit stream (group g at bit g*M).
+ *     slot), little-endian bit stream (group g at bit g*M); for M = 8 one
+ *     mask byte per chunk.
  * Slots are the group's nonzero positions plus, if fewer than N, its lowest
- * zero positions.  Buffer = d_out code rows, then d_out index rows.
+ * zero positions.  Buffer = d_out code rows, then d_out index rows; sbl_pack
+ * writes the padding as zero bytes.
  * A group with more than N nonzeros latches SBL_ERR_DEVICE_CHECK.
  * ---------------------------------------------------------------------- */
 size_t sbl_packed_bytes(int d_out, int d_in, int N, int M);
