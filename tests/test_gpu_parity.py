@@ -146,6 +146,38 @@ def test_gamma_exact_on_extreme_magnitudes(lib):
     assert np.array_equal(L.W_eff.cpu().numpy(), weff)
 
 
+@pytest.mark.parametrize("accumulate", [False, True])
+def test_empty_token_batch(lib, variant, accumulate):
+    """T = 0, an empty batch: the weight side still runs; quantisation, the
+    forward product and dX have no rows to write; dW is the empty sum (all
+    zeros, written over whatever the buffer held) or, when accumulating, the
+    incoming gradient unchanged."""
+    from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer, act_quant
+    d_out, d_in, N, M = 264, 400, 6, 8
+    w = synth.trimodal_weight(d_out, d_in, seed=5, tensor_id=0)
+    x = synth.activations(0, d_in, seed=5, tensor_id=1)
+    dy = synth.grad_output(0, d_out, seed=5, tensor_id=2)
+    L = SparseBitLinearLayer(_dev(w), N, M, keep_mask=True)
+    L.weight_step()
+    X = _dev(x)
+    Xq = torch.empty(0, d_in, dtype=torch.int8, device="cuda")
+    amax = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+    act_quant(X, Xq, amax)
+    Y = torch.empty(0, d_out, dtype=torch.float32, device="cuda")
+    L.forward(Xq, amax, Y)
+    dX = torch.empty(0, d_in, dtype=torch.float32, device="cuda")
+    before = 0.25 if accumulate else float("nan")
+    dW = torch.full((d_out, d_in), before, dtype=torch.float32, device="cuda")
+    L.backward(_dev(dy), X, dX, dW, accumulate_dW=accumulate)
+    lib.sbl_check()
+    torch.cuda.synchronize()
+    weff, gamma, _ = oracle.effective_weight(synth.bits(w), N, M)
+    assert np.array_equal(L.W_eff.cpu().numpy(), weff)
+    assert L.gamma.item() == float(gamma)
+    assert amax.item() == -1.0  # nothing written for an empty batch
+    assert torch.all(dW == (0.25 if accumulate else 0.0)).item()
+
+
 def test_dw_split_k_and_accumulate(lib, variant):
     """Small d_out (k/v-like) takes the split-K path with atomics; the
     accumulate flag adds into an existing gradient."""
