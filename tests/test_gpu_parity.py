@@ -146,6 +146,32 @@ def test_gamma_exact_on_extreme_magnitudes(lib):
     assert np.array_equal(L.W_eff.cpu().numpy(), weff)
 
 
+@pytest.mark.parametrize("kind", ["zero", "constant_magnitude"])
+def test_degenerate_weights(lib, kind):
+    """An all-zero weight (gamma = 0: every weight is divided by eps alone and
+    rounds to 0) and a weight of one magnitude with random signs (every group
+    is a full tie, so the lowest N positions are kept, and every kept weight
+    is +-1).  The whole path matches the oracle."""
+    d_out, d_in, T, N, M = 136, 400, 70, 6, 8
+    if kind == "zero":
+        w = torch.zeros(d_out, d_in, dtype=torch.bfloat16)
+    else:
+        g = torch.Generator().manual_seed(11)
+        sign = torch.randint(0, 2, (d_out, d_in), generator=g) * 2 - 1
+        w = (sign.float() * 0.375).to(torch.bfloat16)
+    x = synth.activations(T, d_in, seed=6, tensor_id=1)
+    dy = synth.grad_output(T, d_out, seed=6, tensor_id=2)
+    gl, ref = _full_parity(lib, w, x, dy, N, M)
+    if kind == "zero":
+        assert gl.L.gamma.item() == 0.0
+        assert not gl.Y.cpu().numpy().any()
+    else:
+        keep = _unpack_mask(gl.L.mask_bits.cpu().numpy()).reshape(d_out, d_in // M, M)
+        assert keep[:, :, :N].all() and not keep[:, :, N:].any()
+        assert np.array_equal(np.abs(gl.L.W_eff.cpu().numpy()).reshape(d_out, d_in // M, M)[:, :, :N],
+                              np.ones((d_out, d_in // M, N), np.int8))
+
+
 @pytest.mark.parametrize("accumulate", [False, True])
 def test_empty_token_batch(lib, variant, accumulate):
     """T = 0, an empty batch: the weight side still runs; quantisation, the
