@@ -26,7 +26,8 @@
  *     IEEE bfloat16 bit patterns (uint16 per element).
  *   - Every pointer must be 16-byte aligned.  d_in must be a multiple of 16
  *     and of M; d_out must be a multiple of 8.  T (tokens) may be any value
- *     >= 0; T = 0 is a no-op.
+ *     >= 0; with T = 0 no token row is written (sbl_backward's dW, a sum
+ *     over tokens, is then zero-filled, or left as it is when accumulating).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Every call only enqueues work on `stream` and returns; it
  *     never synchronises.
@@ -263,7 +264,8 @@ sbl_status sbl_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff,
  * together have at most four 256 x 256 output tiles per pair of SMs (short
  * token batches, such as a prefill of a few hundred tokens) they run in one
  * launch, which pays the fixed start-up cost once; larger ones run one launch
- * each.  Same citation as sbl_forward.
+ * each (as do all products under sbl_set_gemm_variant(1)).  Same citation as
+ * sbl_forward.
  *   problems  HOST array of `count` descriptors (read before the call
  *             returns; the pointers inside are device pointers); each is
  *             validated as sbl_forward validates its arguments. */
