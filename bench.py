@@ -566,9 +566,9 @@ def run_normquant(args):
 def run_optimizer(args):
     """The optimizer step over the 3B layer set (7 projections, 77 M weights):
     sbl_grad_sqnorm over every dW (the global clip norm), then one
-    sbl_adamw_step per projection (AdamW on the bf16 master weight, clip at
-    max_norm 1, the next step's exact gamma pass, the mask flip count, then
-    the ternary pass).  Also the same with an fp32 master copy.  Inputs:
+    sbl_adamw_step per projection on three side streams (AdamW on the bf16
+    master weight, clip at max_norm 1, the next step's exact gamma pass, the
+    mask flip count, then the ternary pass).  Also the same with an fp32 master copy.  Inputs:
     trimodal bf16 weights, synthetic fp32 gradients and moments (synth),
     1.3 GB or more resident, far larger than L2.  CUDA events on the
     launching stream."""
@@ -604,13 +604,29 @@ def run_optimizer(args):
         for q in projs:
             sbl.sbl_grad_sqnorm(q["dW"], q["dW"].numel(), sumsq, q["ws"], q["ws_bytes"], stream)
 
+    # The projections' steps are independent once the global norm is known
+    # (each has its own workspace; the flip counter is added atomically), so
+    # they run on three side streams, largest first, as the training step runs
+    # its weight steps; sbl_grad_sqnorm adds into one sum and stays in order on
+    # the main stream.
+    side = [torch.cuda.Stream() for _ in range(3)]
+    by_size = sorted(projs, key=lambda q: -q["p"].d_out * q["p"].d_in)
+
     def adamw(master32):
         state["t"] += 1
-        for q in projs:
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        for sd in side:
+            sd.wait_event(fork)
+        for i, q in enumerate(by_size):
             p = q["p"]
             sbl.sbl_adamw_step(q["W"], q["W32"] if master32 else None, q["dW"], q["m"], q["v"], p.d_out, p.d_in,
                                N, M, 1e-5, 0.9, 0.95, 1e-5, 0.1, state["t"], sumsq, 1.0, q["weff"], q["weff16"],
-                               q["bits"], q["gamma"], flips, q["ws"], q["ws_bytes"], stream)
+                               q["bits"], q["gamma"], flips, q["ws"], q["ws_bytes"], side[i % len(side)])
+        for sd in side:
+            join = torch.cuda.Event()
+            join.record(sd)
+            stream.wait_event(join)
 
     # algorithmic bytes per weight: adamw launch (W 2+2 or W32 4+4 and the bf16 W write, dW 4, m 4+4,
     # v 4+4, old mask 1/8) + ternary pass (W 2, W_eff 1, W_eff bf16 2, mask 1/8)
