@@ -263,9 +263,11 @@ sbl_status sbl_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff,
  * problem i is exactly sbl_forward on its own buffers.  While the products
  * together have at most four 256 x 256 output tiles per pair of SMs (short
  * token batches, such as a prefill of a few hundred tokens) they run in one
- * launch, which pays the fixed start-up cost once; larger ones run one launch
- * each (as do all products under sbl_set_gemm_variant(1)).  Same citation as
- * sbl_forward.
+ * launch, which pays the fixed start-up cost once; inside it a product whose
+ * K is at least twice the group's shortest is split in K (exact integer
+ * partial sums added into Y, then scaled in place by a second pass, so Y is
+ * written twice).  Larger groups run one launch per product (as do all
+ * products under sbl_set_gemm_variant(1)).  Same citation as sbl_forward.
  *   problems  HOST array of `count` descriptors (read before the call
  *             returns; the pointers inside are device pointers); each is
  *             validated as sbl_forward validates its arguments. */

@@ -26,6 +26,7 @@
 //     latched error instead of hanging.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -1035,6 +1036,33 @@ cudaError_t launch_forward_group(const FwdProblemDev* probs, int count, cudaStre
         order[k - 1] = tmp;
       }
     if (n == 0) continue;
+    // A product whose K loop is much longer than the group's shortest one is
+    // cut into K splits of about that length, so its tiles do not set the
+    // launch's length alone.  The splits add their exact integer sums into a
+    // zeroed Y (|acc| <= 128 * d_in < 2^24 keeps every fp32 partial exact) and
+    // a pass after the launch scales Y in place, as the single-product split.
+    int kb_min = 1 << 30;
+    for (int i = 0; i < n; ++i) kb_min = std::min(kb_min, (probs[order[i]].d_in + 127) / 128);
+    int split_of[kFwdGroup];
+    for (int i = 0; i < n; ++i) {
+      const FwdProblemDev& q = probs[order[i]];
+      const int KB = (q.d_in + 127) / 128;
+      int splits = 1;
+      if (KB >= 2 * kb_min && q.d_in < (1 << 17)) {
+        splits = (KB + kb_min - 1) / kb_min;
+        if (splits > KB / 4) splits = KB / 4;  // at least four K blocks per split
+        if (splits < 1) splits = 1;
+      }
+      if (splits > 1) {
+        const int kbs = (KB + splits - 1) / splits;
+        splits = (KB + kbs - 1) / kbs;
+      }
+      split_of[i] = splits;
+      if (splits > 1) {
+        const cudaError_t e = cudaMemsetAsync(q.Y, 0, sizeof(float) * static_cast<size_t>(q.T) * q.d_out, stream);
+        if (e != cudaSuccess) return e;
+      }
+    }
     PairGroup<kFwdGroup> grp{};
     int total = 0;
     for (int i = 0; i < n; ++i) {
@@ -1046,7 +1074,9 @@ cudaError_t launch_forward_group(const FwdProblemDev* probs, int count, cudaStre
       a.M = q.T;
       a.N = q.d_out;
       a.K = q.d_in;
-      a.kb_per_split = (q.d_in + 127) / 128;
+      const int KB = (q.d_in + 127) / 128;
+      a.kb_per_split = (KB + split_of[i] - 1) / split_of[i];
+      a.atomic_i32 = split_of[i] > 1 ? 1 : 0;
       a.out = q.Y;
       a.ldo = q.d_out;
       a.acc_out = q.acc;
@@ -1056,8 +1086,8 @@ cudaError_t launch_forward_group(const FwdProblemDev* probs, int count, cudaStre
       Sched& sc = grp.sched[i];
       sc.Mt = (q.T + 255) / 256;
       sc.Nt = (q.d_out + C::BN - 1) / C::BN;
-      sc.splits = 1;
-      sc.total = sc.Mt * sc.Nt;
+      sc.splits = split_of[i];
+      sc.total = sc.Mt * sc.Nt * sc.splits;
       sc.GM = pick_strip(sc.Mt, sc.Nt, num_sms / 2, static_cast<double>(q.T) * q.d_in,
                          static_cast<double>(q.d_out) * q.d_in);
       grp.item_start[i] = total;
@@ -1073,6 +1103,17 @@ cudaError_t launch_forward_group(const FwdProblemDev* probs, int count, cudaStre
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, 2 * pairs, C::THREADS, C::SMEM_BYTES, stream, grp, PackedB{});
     if (e != cudaSuccess) return e;
+    for (int i = 0; i < n; ++i) {
+      if (split_of[i] == 1) continue;
+      const FwdProblemDev& q = probs[order[i]];
+      const size_t n4 = static_cast<size_t>(q.T) * q.d_out / 4;
+      size_t blocks = (n4 + 255) / 256;
+      if (blocks > static_cast<size_t>(num_sms) * 8) blocks = static_cast<size_t>(num_sms) * 8;
+      fwd_split_finalize_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+          reinterpret_cast<float4*>(q.Y), reinterpret_cast<int4*>(q.acc), q.amax, q.gamma, q.d_out, n4);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
   }
   return cudaSuccess;
 }
