@@ -17,9 +17,9 @@
 // HBM bound: X is read once (2 B per element), Xq written once (1 B) and,
 // when requested, the normalised row xn (2 B, the bf16 input of the dW
 // product).  Compared with a separate norm kernel feeding act_quant this
-// saves one read and one write of X.  Each row lives in registers (up to
-// 8 x 16 bytes per thread, TPR threads per row); longer rows re-read their
-// tail from L2.
+// saves one read and one write of X.  Each row lives in registers (8, or 6
+// for rows of 256 threads that fit, x 16 bytes per thread, TPR threads per
+// row); longer rows re-read their tail from L2.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -130,7 +130,7 @@ __device__ __forceinline__ V row_reduce(V x, V* scratch, int rib, bool is_max) {
   return x;
 }
 
-template <int TPR>
+template <int TPR, int VPT>
 __global__ void __launch_bounds__(kNqThreads) norm_quant_kernel(const uint4* __restrict__ X,
                                                                 const uint4* __restrict__ G, float eps, int T,
                                                                 int nv, uint4* __restrict__ Xn,
@@ -152,29 +152,29 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_kernel(const uint4* __r
     const long long row = base + rib;
     const bool active = row < T;
     const uint4* xr = X + (active ? row : static_cast<long long>(T) - 1) * static_cast<long long>(nv);
-    uint4 v[kNqVpt];
+    uint4 v[VPT];
     double ss = 0.0;
 #pragma unroll
-    for (int k = 0; k < kNqVpt; ++k) {
+    for (int k = 0; k < VPT; ++k) {
       const int idx = tr + k * TPR;
       v[k] = idx < nv ? __ldg(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int k = 0; k < kNqVpt; ++k) ss = sumsq8(v[k], ss);
-    for (int idx = tr + kNqVpt * TPR; idx < nv; idx += TPR) ss = sumsq8(__ldg(xr + idx), ss);
+    for (int k = 0; k < VPT; ++k) ss = sumsq8(v[k], ss);
+    for (int idx = tr + VPT * TPR; idx < nv; idx += TPR) ss = sumsq8(__ldg(xr + idx), ss);
     ss = row_reduce<TPR, double>(ss, s_sum, rib, false);
     const float vv = static_cast<float>(ss / static_cast<double>(d) + static_cast<double>(eps));
     const float r = __fdiv_rn(1.0f, __fsqrt_rn(vv));
 
     uint32_t mx = 0u;
 #pragma unroll
-    for (int k = 0; k < kNqVpt; ++k) {
+    for (int k = 0; k < VPT; ++k) {
       const int idx = tr + k * TPR;
       const uint4 gk = idx < nv ? __ldg(G + idx) : make_uint4(0u, 0u, 0u, 0u);
       v[k] = norm8(v[k], gk, r);
       mx = __vmaxu2(mx, maxmag8(v[k]));
     }
-    for (int idx = tr + kNqVpt * TPR; idx < nv; idx += TPR)
+    for (int idx = tr + VPT * TPR; idx < nv; idx += TPR)
       mx = __vmaxu2(mx, maxmag8(norm8(__ldg(xr + idx), __ldg(G + idx), r)));
     mx = max(mx & 0xFFFFu, mx >> 16);
     mx = row_reduce<TPR, uint32_t>(mx, s_max, rib, true);
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_kernel(const uint4* __r
     uint2* qr = Xq + row * static_cast<long long>(nv);
     uint4* nr = Xn != nullptr ? Xn + row * static_cast<long long>(nv) : nullptr;
 #pragma unroll
-    for (int k = 0; k < kNqVpt; ++k) {
+    for (int k = 0; k < VPT; ++k) {
       const int idx = tr + k * TPR;
       const uint2 q = quant8(v[k], sc);
       if (active && idx < nv) {
@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_kernel(const uint4* __r
       }
     }
     if (active) {
-      for (int idx = tr + kNqVpt * TPR; idx < nv; idx += TPR) {
+      for (int idx = tr + VPT * TPR; idx < nv; idx += TPR) {
         const uint4 u = norm8(__ldg(xr + idx), __ldg(G + idx), r);
         qr[idx] = quant8(u, sc);
         if (nr != nullptr) nr[idx] = u;
@@ -202,17 +202,29 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_kernel(const uint4* __r
   }
 }
 
-template <int TPR>
-cudaError_t launch_nq(const void* X, const void* g, float eps, int T, int nv, void* Xn, int8_t* Xq, float* amax,
-                      cudaStream_t stream, int num_sms) {
+template <int TPR, int VPT>
+cudaError_t launch_nq_v(const void* X, const void* g, float eps, int T, int nv, void* Xn, int8_t* Xq, float* amax,
+                        cudaStream_t stream, int num_sms) {
   constexpr int RPB = kNqThreads / TPR;
   long long blocks = (static_cast<long long>(T) + RPB - 1) / RPB;
   const long long cap = static_cast<long long>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
-  norm_quant_kernel<TPR><<<static_cast<unsigned>(blocks), kNqThreads, 0, stream>>>(
+  norm_quant_kernel<TPR, VPT><<<static_cast<unsigned>(blocks), kNqThreads, 0, stream>>>(
       static_cast<const uint4*>(X), static_cast<const uint4*>(g), eps, T, nv, static_cast<uint4*>(Xn),
       reinterpret_cast<uint2*>(Xq), amax);
   return cudaGetLastError();
+}
+
+// Vectors held in registers per thread.  A row of 256 threads that fits in
+// 6 (such as 1376 vectors, d = 11008) holds 6 instead of 8, so it runs no
+// arithmetic on two zero-filled vectors past its end; narrower rows keep 8.
+template <int TPR>
+cudaError_t launch_nq(const void* X, const void* g, float eps, int T, int nv, void* Xn, int8_t* Xq, float* amax,
+                      cudaStream_t stream, int num_sms) {
+  if constexpr (TPR == 256) {
+    if (nv <= 6 * TPR) return launch_nq_v<TPR, 6>(X, g, eps, T, nv, Xn, Xq, amax, stream, num_sms);
+  }
+  return launch_nq_v<TPR, kNqVpt>(X, g, eps, T, nv, Xn, Xq, amax, stream, num_sms);
 }
 
 }  // namespace
