@@ -93,6 +93,47 @@ def test_host_validation_without_gpu(cl):
     assert cl.sbl_forward(al, al, al, al, 0, 16, 8, al, None, None) == 0
 
 
+def test_group_and_variant_validation_without_gpu(cl):
+    """Grouped calls check every descriptor on the host; the kernel-variant
+    selectors accept only their documented values."""
+    from semi_structured_sparsity_step_b200 import _binding as B
+    al = 1 << 12
+    assert cl.sbl_set_gemm_variant(2) == 1
+    assert cl.sbl_set_gemm_variant(-1) == 1
+    assert cl.sbl_set_gemv_variant(2) == 1
+    assert cl.sbl_set_gemm_variant(0) == 0 and cl.sbl_set_gemv_variant(0) == 0
+
+    def fwd(*problems):
+        arr = (B.ForwardProblem * max(1, len(problems)))()
+        for i, q in enumerate(problems):
+            arr[i] = B.ForwardProblem(*q)
+        return cl.sbl_forward_group(ctypes.cast(arr, ctypes.c_void_p), len(problems), None)
+
+    good = (al, al, al, al, 4, 16, 8, al, None)
+    assert cl.sbl_forward_group(None, -1, None) == 1
+    assert cl.sbl_forward_group(None, 1, None) == 1
+    assert cl.sbl_forward_group(None, 0, None) == 0
+    assert fwd(good, (al, al, al, al, 4, 20, 8, al, None)) == 2   # d_in % 16 in the second problem
+    assert fwd(good, (al, al, al, al, -1, 16, 8, al, None)) == 2  # negative T
+    assert fwd(good, (al, None, al, al, 4, 16, 8, al, None)) == 1
+    assert fwd(good, (al, al, al, al + 2, 4, 16, 8, al, None)) == 3  # gamma not 4-byte aligned
+    assert fwd((al, al, al, al, 0, 16, 8, al, None)) == 0         # only empty work: no device needed
+
+    def gemv(batch, *problems, N=6, M=8):
+        arr = (B.GemvProblem * max(1, len(problems)))()
+        for i, q in enumerate(problems):
+            arr[i] = B.GemvProblem(*q)
+        return cl.sbl_gemv_packed_group(arr, len(problems), batch, N, M, None)
+
+    gp = (al, al, al, al, al, 16, 8)
+    assert gemv(17, gp) == 2
+    assert gemv(1, gp, N=5, M=6) == 1
+    assert gemv(1, gp, (al, al, al, al, al, 24, 8)) == 2  # d_in % 16
+    assert gemv(1, gp, (None, al, al, al, al, 16, 8)) == 1
+    assert gemv(1, gp, (al + 8, al, al, al, al, 16, 8)) == 3
+    assert gemv(0, gp) == 0
+
+
 def test_packed_bytes_matches_format(cl):
     import oracle
     for (d_out, d_in, N, M) in [(8, 16, 6, 8), (24, 272, 2, 4), (2048, 11008, 6, 8), (16, 64, 8, 8)]:
