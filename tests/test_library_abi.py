@@ -126,6 +126,8 @@ def test_group_and_variant_validation_without_gpu(cl):
         return cl.sbl_gemv_packed_group(arr, len(problems), batch, N, M, None)
 
     gp = (al, al, al, al, al, 16, 8)
+    assert cl.sbl_gemv_dense2_group(None, 1, 17, None) == 2
+    assert cl.sbl_gemv_dense2_group(None, 1, 1, None) == 1
     assert gemv(17, gp) == 2
     assert gemv(1, gp, N=5, M=6) == 1
     assert gemv(1, gp, (al, al, al, al, al, 24, 8)) == 2  # d_in % 16
@@ -139,3 +141,46 @@ def test_packed_bytes_matches_format(cl):
     for (d_out, d_in, N, M) in [(8, 16, 6, 8), (24, 272, 2, 4), (2048, 11008, 6, 8), (16, 64, 8, 8)]:
         assert cl.sbl_packed_bytes(d_out, d_in, N, M) == oracle.packed_layout(d_out, d_in, N, M)[2]
     assert cl.sbl_packed_bytes(8, 24, 6, 8) == 0  # invalid shape
+
+
+def test_remaining_entry_points_validate_on_the_host(cl):
+    """Every other entry point rejects bad flags, N:M, shapes, null or
+    misaligned pointers and short buffers before it needs a device, and
+    treats empty work as done."""
+    al = 1 << 12
+    ws = 1 << 20
+    # mask from the quantised weight: unknown flag bits
+    assert cl.sbl_mask_quant_ex(al, 8, 16, 6, 8, 2, al, None, None, al, al * 4, ws, None) == 1
+    # dW (.) M
+    assert cl.sbl_mask_grad(al, al, 8, 20, None) == 2
+    assert cl.sbl_mask_grad(None, al, 8, 16, None) == 1
+    assert cl.sbl_mask_grad(al + 4, al, 8, 16, None) == 3
+    assert cl.sbl_mask_grad(al, al, 0, 16, None) == 0
+    # forward from the packed format
+    assert cl.sbl_forward_packed(al, al, al, al, 4, 16, 8, 5, 6, al, None, None) == 1
+    assert cl.sbl_forward_packed(al, al, al, al, -1, 16, 8, 6, 8, al, None, None) == 2
+    assert cl.sbl_forward_packed(al, al, None, al, 4, 16, 8, 6, 8, al, None, None) == 1
+    assert cl.sbl_forward_packed(al, al, al, al, 0, 16, 8, 6, 8, al, None, None) == 0
+    # unpack
+    assert cl.sbl_unpack(al, 8, 16, 9, 8, al, None) == 1
+    assert cl.sbl_unpack(al, 8, 16, 6, 8, None, None) == 1
+    assert cl.sbl_unpack(al, 8, 16, 6, 8, al + 8, None) == 3
+    # 2:4 compression and the sparse forward
+    assert cl.sbl_compress24(al, 8, 16, None, 1 << 20, None) == 1
+    assert cl.sbl_compress24(al, 8, 16, al, 16, None) == 5
+    assert cl.sbl_forward_sparse24(al, al, al, al, -1, 16, 8, al, None, None) == 2
+    assert cl.sbl_forward_sparse24(al, al, al, al + 2, 4, 16, 8, al, None, None) == 3
+    assert cl.sbl_forward_sparse24(al, al, al, al, 0, 16, 8, al, None, None) == 0
+    # dense 2-bit layout
+    assert cl.sbl_pack_dense2(al, 8, 16, al, 4, None) == 5
+    assert cl.sbl_pack_dense2(None, 8, 16, al, 1 << 20, None) == 1
+    # fused norm + quantiser
+    assert cl.sbl_rmsnorm_act_quant(al, al, 0.0, 4, 16, None, al, al, None) == 1
+    assert cl.sbl_rmsnorm_act_quant(al, None, 1e-6, 4, 16, None, al, al, None) == 1
+    assert cl.sbl_rmsnorm_act_quant(al, al, 1e-6, 4, 16, al + 8, al, al, None) == 3
+    assert cl.sbl_rmsnorm_act_quant(al, al, 1e-6, 0, 16, None, al, al, None) == 0
+    # backward
+    assert cl.sbl_backward(al, al, al, al, -1, 16, 8, al, al, 0, None, 0, None) == 2
+    assert cl.sbl_backward(al, al, None, al, 4, 16, 8, al, None, 0, None, 0, None) == 1
+    assert cl.sbl_backward(al, al, al, al, 4, 16, 8, None, al + 4, 0, None, 0, None) == 3
+    assert cl.sbl_backward(al, al, al, al, 4, 16, 8, None, None, 0, None, 0, None) == 0
