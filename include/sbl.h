@@ -83,6 +83,17 @@ sbl_status sbl_set_gemm_variant(int variant);
  * sums, the same scaling).  Same threading caveat as sbl_set_gemm_variant. */
 sbl_status sbl_set_gemv_variant(int variant);
 
+/* Failure-detection self-test.  Every spin-wait of this library gives up
+ * after a time limit, latches SBL_ERR_TIMEOUT in the device's error word and
+ * returns, so a lost signal ends as an error status instead of a hung
+ * device.  This call launches one kernel that takes that path on purpose: it
+ * waits on a barrier phase that nothing completes for limit_us microseconds
+ * (1..1000000), then latches the timeout and exits.  The next sbl_check on
+ * this device returns SBL_ERR_TIMEOUT and clears it; the CUDA context stays
+ * usable.  The pages have no counterpart: it checks the library's own error
+ * path. */
+sbl_status sbl_selftest_wait_timeout(unsigned limit_us, void* stream);
+
 /* Synchronise `stream`, then return (and clear) the first error latched by a
  * kernel of this library on the current device since the previous check;
  * SBL_OK if none.  Also reports a pending CUDA error as SBL_ERR_CUDA. */

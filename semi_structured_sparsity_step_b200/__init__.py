@@ -13,8 +13,8 @@ from ._binding import (  # noqa: F401
     sbl_gemv_packed, sbl_gemv_packed_group, sbl_grad_sqnorm, sbl_mask_grad, sbl_mask_quant,
     sbl_mask_quant_ex, sbl_mask_quant_noalloc, sbl_mask_quant_noalloc_scratch_bytes,
     sbl_mask_quant_workspace_bytes, sbl_pack, sbl_pack_dense2, sbl_packed_bytes,
-    sbl_rmsnorm_act_quant, sbl_set_gemm_variant, sbl_set_gemv_variant, sbl_status_string,
-    sbl_unpack, sbl_version,
+    sbl_rmsnorm_act_quant, sbl_selftest_wait_timeout, sbl_set_gemm_variant, sbl_set_gemv_variant,
+    sbl_status_string, sbl_unpack, sbl_version,
 )
 
 __all__ = [
@@ -24,6 +24,7 @@ __all__ = [
     "sbl_gemv_packed", "sbl_gemv_packed_group", "sbl_grad_sqnorm", "SBL_MASK_FROM_QUANTISED",
     "sbl_mask_grad", "sbl_mask_quant", "sbl_mask_quant_ex", "sbl_mask_quant_noalloc",
     "sbl_mask_quant_noalloc_scratch_bytes", "sbl_mask_quant_workspace_bytes", "sbl_pack",
-    "sbl_pack_dense2", "sbl_packed_bytes", "sbl_rmsnorm_act_quant", "sbl_set_gemm_variant",
-    "sbl_set_gemv_variant", "sbl_status_string", "sbl_unpack", "sbl_version", "SblError",
+    "sbl_pack_dense2", "sbl_packed_bytes", "sbl_rmsnorm_act_quant", "sbl_selftest_wait_timeout",
+    "sbl_set_gemm_variant", "sbl_set_gemv_variant", "sbl_status_string", "sbl_unpack",
+    "sbl_version", "SblError",
 ]

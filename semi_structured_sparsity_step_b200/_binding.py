@@ -36,6 +36,7 @@ SIGNATURES = {
     "sbl_version": (_c_int, []),
     "sbl_set_gemv_variant": (_c_int, [_c_int]),
     "sbl_check": (_c_int, [_vp]),
+    "sbl_selftest_wait_timeout": (_c_int, [ctypes.c_uint, _vp]),
     "sbl_set_gemm_variant": (_c_int, [_c_int]),
     "sbl_mask_quant_workspace_bytes": (_c_size, [_c_int, _c_int]),
     "sbl_mask_quant": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
@@ -142,6 +143,10 @@ def sbl_set_gemv_variant(variant: int) -> None:
 
 def sbl_check(stream=None) -> None:
     _call("sbl_check", _stream(stream))
+
+
+def sbl_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    _call("sbl_selftest_wait_timeout", int(limit_us), _stream(stream))
 
 
 def sbl_mask_quant_workspace_bytes(d_out: int, d_in: int) -> int:

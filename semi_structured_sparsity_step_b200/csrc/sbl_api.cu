@@ -107,6 +107,15 @@ sbl_status sbl_set_gemv_variant(int variant) {
   return SBL_OK;
 }
 
+sbl_status sbl_selftest_wait_timeout(unsigned limit_us, void* stream) {
+  if (limit_us == 0u || limit_us > 1000000u) return SBL_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  const sbl_status st = current_device(&d);
+  if (st != SBL_OK) return st;
+  return from_cuda(launch_wait_timeout_selftest(static_cast<uint64_t>(limit_us) * 1000ull,
+                                                static_cast<cudaStream_t>(stream), d->err));
+}
+
 sbl_status sbl_check(void* stream) {
   DeviceInfo* d = nullptr;
   sbl_status st = current_device(&d);

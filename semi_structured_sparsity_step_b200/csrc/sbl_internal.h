@@ -112,6 +112,8 @@ struct GemvProblemDev {
 extern int g_gemv_variant;
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
                               cudaStream_t stream, int num_sms, uint32_t* err, bool dense2);
+// Failure-detection self-test: one bounded wait that runs out (selftest.cu).
+cudaError_t launch_wait_timeout_selftest(uint64_t limit_ns, cudaStream_t stream, uint32_t* err);
 cudaError_t launch_gemv_direct(const GemvProblemDev* probs, int count, int batch, int N, int M,
                                cudaStream_t stream, int num_sms, uint32_t* err, bool dense2);
 size_t dense2_row_bytes(int d_in);

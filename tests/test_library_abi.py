@@ -149,6 +149,9 @@ def test_remaining_entry_points_validate_on_the_host(cl):
     treats empty work as done."""
     al = 1 << 12
     ws = 1 << 20
+    # failure-detection self-test: the wait limit must be 1 us .. 1 s
+    assert cl.sbl_selftest_wait_timeout(0, None) == 1
+    assert cl.sbl_selftest_wait_timeout(2000000, None) == 1
     # mask from the quantised weight: unknown flag bits
     assert cl.sbl_mask_quant_ex(al, 8, 16, 6, 8, 2, al, None, None, al, al * 4, ws, None) == 1
     # dW (.) M
