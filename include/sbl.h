@@ -38,6 +38,11 @@
  *     nonzeros in a group) are latched in a device word and returned by the
  *     next sbl_check() on that device.
  *   - No call throws or aborts across the ABI.
+ *   - The library caches per-device state the first time a device is used
+ *     (the address of its device error word, of sbl_mask_quant_noalloc's
+ *     scratch array, kernel attributes).  cudaDeviceReset() destroys the
+ *     context that state points into: after resetting a device, do not call
+ *     this library on that device again in the same process.
  */
 #ifndef SBL_H_
 #define SBL_H_
@@ -218,7 +223,8 @@ sbl_status sbl_adamw_step(void* W, float* W32, const float* dW, float* m, float*
  *     larger W returns SBL_ERR_SHAPE without launching anything.
  *   - The first call on a device looks up the scratch array's device address
  *     (once per device, with that device current) and caches it; make that
- *     first call before any stream capture.
+ *     first call before any stream capture.  A cudaDeviceReset() leaves the
+ *     cached address stale (see the conventions above).
  *   - All calls on a device share the one scratch array.  Each call clears
  *     the part that must start at zero, but calls that overlap on the GPU
  *     (different streams, or different host threads without ordering) race

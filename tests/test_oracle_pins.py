@@ -299,6 +299,78 @@ def test_forward_output_error_bound():
     assert np.abs(r["y"] - ref).max() < 0.05 * np.abs(ref).max()
 
 
+U32 = Fraction(1, 1 << 24)   # unit roundoff of fp32, round to nearest
+
+
+def _ulp_close(got: float, want: Fraction, n_roundings: int) -> bool:
+    """|got - want| <= n rounding errors of fp32 relative to |want|."""
+    return abs(Fraction(float(got)) - want) <= n_roundings * U32 * abs(want)
+
+
+def test_forward_out_is_the_exact_scaled_product():
+    """Summary, Algorithm 1 step (6) ("s absorbs the quantisation scales")
+    with 前置知识's absmax scale 127/max|x|: y = acc * gamma * amax / 127.
+    Checked against exact rationals: the oracle's three fp32 roundings
+    (amax/127, gamma*(.), acc*(.)) leave at most 3 ulps.  A slip of the
+    level (128 for 127), a dropped or squared gamma, or an inverted amax is
+    off by far more than that."""
+    rng = np.random.default_rng(21)
+    T, d_out = 40, 24
+    acc = rng.integers(-(1 << 20), 1 << 20, size=(T, d_out)).astype(np.int32)
+    acc[0, :3] = [0, 1, -1]
+    amax = np.exp(rng.uniform(np.log(1e-5), np.log(60.0), size=T)).astype(np.float32)
+    amax[:4] = [np.float32(1e-5), 3.0, 0.3125, 2.75]     # floor and non-powers of two
+    for gamma in [np.float32(0.0234375), np.float32(rng.uniform(1e-3, 0.1)), np.float32(0.0)]:
+        y = oracle.forward_out(acc, gamma, amax)
+        assert y.dtype == np.float32
+        for t in range(T):
+            for o in range(d_out):
+                want = Fraction(int(acc[t, o])) * Fraction(float(gamma)) * Fraction(float(amax[t])) / 127
+                assert _ulp_close(y[t, o], want, 3), (t, o, y[t, o], float(want))
+
+
+def test_forward_hand_built_layer_exact():
+    """The whole forward on inputs whose every intermediate is known by hand
+    (summary, Algorithm 1 steps (2)-(6); 前置知识).  W has one magnitude
+    c = 3/128 with hand-set signs, so gamma = c exactly, every code is the
+    sign, and at 6:8 the first six positions of each group are kept (all
+    ties).  The int8 codes are round-half-even of x * 127 / amax in exact
+    arithmetic (the inputs avoid .5 boundaries), and the expected y is the
+    exact rational sum(xq * W_eff) * c * amax / 127."""
+    c = Fraction(3, 128)
+    d_in = 16
+    signs = np.array([[1, -1, 1, 1, -1, -1, 1, -1, -1, 1, 1, -1, 1, 1, -1, 1],
+                      [-1, -1, -1, 1, 1, 1, -1, 1, 1, 1, -1, -1, 1, -1, 1, 1],
+                      [1, 1, 1, 1, 1, 1, 1, 1, -1, -1, -1, -1, -1, -1, -1, -1]], np.int64)
+    w = _bf16((signs * float(c)).tolist())
+    xs = [[3.0, -1.25, 0.5, 2.0, -0.75, 0.0, 1.75, -2.5, 0.25, -3.0, 1.0, 0.125, -1.625, 2.25, -0.375, 0.625],
+          [0.3125, -0.1875, 0.0625, 0.25, -0.3125, 0.125, 0.0, -0.09375, 0.140625, 0.03125, -0.21875, 0.28125,
+           -0.046875, 0.1875, -0.25, 0.109375],
+          [2.75, 1.4375, -0.6875, 2.0, -2.75, 0.5, 1.125, -1.875, 0.875, -0.25, 2.5, -1.0, 0.1875, -2.125, 1.625,
+           0.75]]
+    x = _bf16(xs)
+    r = oracle.forward(x, w, 6, 8)
+    assert Fraction(float(r["gamma"])) == c
+    keep = np.tile(np.array([1, 1, 1, 1, 1, 1, 0, 0], np.int64), d_in // 8)
+    weff = signs * keep[None, :]
+    assert np.array_equal(r["weff"], weff)
+    for t, row in enumerate(xs):
+        amax = max(abs(Fraction(v)) for v in row)
+        assert Fraction(float(r["amax"][t])) == amax
+        xq = []
+        for v in row:
+            q = Fraction(v) * 127 / amax
+            fl = math.floor(q)
+            assert abs((q - fl) - Fraction(1, 2)) > Fraction(1, 1000), "hand input sits on a rounding tie"
+            xq.append(fl + 1 if q - fl > Fraction(1, 2) else fl)
+        assert r["xq"][t].tolist() == xq
+        for o in range(weff.shape[0]):
+            acc = sum(int(a) * int(b) for a, b in zip(xq, weff[o]))
+            assert int(r["acc"][t, o]) == acc
+            want = Fraction(acc) * c * amax / 127
+            assert _ulp_close(r["y"][t, o], want, 3), (t, o, float(r["y"][t, o]), float(want))
+
+
 def test_dense_8of8_is_plain_bitlinear():
     """Summary, 前置知识: with N = M nothing is masked (plain BitNet b1.58)."""
     w = synth.bits(synth.normal_weight(16, 64, seed=12))

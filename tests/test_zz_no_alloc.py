@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -27,9 +28,14 @@ def test_noalloc_matches_workspace_call_on_two_calls_in_a_row(lib):
     assert lib.sbl_mask_quant_noalloc_scratch_bytes() == 7040
     # Two different weights (and shapes) back to back: the second call must not
     # see anything the first left in the shared scratch.
+    # The third weight has d_out * d_in / 8 = 530,448 eight-weight vectors:
+    # not a multiple of 256, and far more than the gamma pass's grid of at most
+    # 592 blocks of 256 threads covers in one sweep.  Its magnitudes (and so
+    # its ternary threshold) differ from the call before it.
     cases = [(synth.trimodal_weight(1024, 2048, seed=21, tensor_id=0), 6, 8),
-             (synth.with_boundary_ties(synth.normal_weight(264, 528, seed=22, tensor_id=1), 2, 4, seed=22), 2, 4)]
-    for w_cpu, N, M in cases:
+             (synth.with_boundary_ties(synth.normal_weight(264, 528, seed=22, tensor_id=1), 2, 4, seed=22), 2, 4),
+             (synth.normal_weight(2056, 2064, seed=23, tensor_id=2) * 3, 6, 8)]
+    for k, (w_cpu, N, M) in enumerate(cases):
         W = w_cpu.cuda()
         d_out, d_in = W.shape
         ref = _outputs(d_out, d_in)
@@ -42,6 +48,12 @@ def test_noalloc_matches_workspace_call_on_two_calls_in_a_row(lib):
         for a, b in zip(ref, got):
             assert torch.equal(a, b)
         assert got[3].item() > 0.0
+        if k == 2:
+            weff, gamma, keep = oracle.effective_weight(synth.bits(w_cpu), N, M)
+            assert got[3].item() == float(gamma)
+            assert np.array_equal(got[0].cpu().numpy(), weff)
+            bits = np.unpackbits(got[2].cpu().numpy(), axis=1, bitorder="little").astype(bool)
+            assert np.array_equal(bits, keep)
 
 
 def test_noalloc_rejects_oversized_weight(lib):
