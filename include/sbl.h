@@ -81,11 +81,15 @@ int sbl_version(void);
 sbl_status sbl_set_gemm_variant(int variant);
 
 /* Select the decode GEMV kernel used by sbl_gemv_packed(_group) and
- * sbl_gemv_dense2_group for all later calls in this process: 0 = each warp
- * streams its own 16-row slices through its own TMA ring in shared memory,
- * long rows cut into k slices (the default), 1 = one block-wide TMA tile
- * ring with producer and epilogue warps.  Results are identical (exact int32
- * sums, the same scaling).  Same threading caveat as sbl_set_gemm_variant. */
+ * sbl_gemv_dense2_group for all later calls in this process: 0 = the
+ * default: the dense 2-bit layout (and the 8:8 format) through small blocks
+ * whose warps fill TMA rings before waiting for the previous kernel, so
+ * consecutive launches overlap; the N:M formats through kernel 2; 1 = one
+ * block-wide TMA tile ring with producer and epilogue warps, 2 = persistent
+ * blocks in which each warp streams its own 16-row slices through its own
+ * TMA ring, for every format.  Results
+ * are identical (exact int32 sums, the same scaling).  Same threading caveat
+ * as sbl_set_gemm_variant. */
 sbl_status sbl_set_gemv_variant(int variant);
 
 /* Failure-detection self-test.  Every spin-wait of this library gives up

@@ -612,10 +612,15 @@ int g_gemv_variant = 0;
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
                               cudaStream_t stream, int num_sms, uint32_t* err, bool dense2) {
   if (batch == 0 || count == 0) return cudaSuccess;
-  if (g_gemv_variant == 0) {
+  if (g_gemv_variant == 0 || g_gemv_variant == 2) {
     for (int c0 = 0; c0 < count; c0 += kGemvMaxGroup) {
       const int cnt = (count - c0) < kGemvMaxGroup ? (count - c0) : kGemvMaxGroup;
-      const cudaError_t e = launch_gemv_direct(probs + c0, cnt, batch, N, M, stream, num_sms, err, dense2);
+      // the dense layout (and the 8:8 format, whose codes plane it is) through
+      // the TMA-fed kernel; the N:M formats through the per-warp ring kernel
+      const bool dense = dense2 || N == M;
+      const cudaError_t e = (g_gemv_variant == 0 && dense)
+                                ? launch_gemv_dense_tma(probs + c0, cnt, batch, stream, num_sms, err)
+                                : launch_gemv_direct(probs + c0, cnt, batch, N, M, stream, num_sms, err, dense2);
       if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -102,7 +102,7 @@ sbl_status sbl_set_gemm_variant(int variant) {
 }
 
 sbl_status sbl_set_gemv_variant(int variant) {
-  if (variant != 0 && variant != 1) return SBL_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 2) return SBL_ERR_INVALID_ARG;
   g_gemv_variant = variant;
   return SBL_OK;
 }

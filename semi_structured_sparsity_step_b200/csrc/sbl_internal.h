@@ -107,8 +107,10 @@ struct GemvProblemDev {
   size_t crow, irow;  // filled in by the launcher
   int rows;           // rows per work unit (16 or 8), filled in by the launcher
 };
-// Decode GEMV kernel: 0 = per-warp streaming (gemv_direct.cu, the default),
-// 1 = block-wide TMA tile ring (pack_gemv.cu).
+// Decode GEMV kernel: 0 = the default (the dense layout through gemv_tma.cu,
+// the N:M formats through gemv_direct.cu), 1 = block-wide TMA tile ring
+// (pack_gemv.cu), 2 = per-warp TMA rings in persistent blocks
+// (gemv_direct.cu) for every format.
 extern int g_gemv_variant;
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
                               cudaStream_t stream, int num_sms, uint32_t* err, bool dense2);
@@ -116,6 +118,10 @@ cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch,
 cudaError_t launch_wait_timeout_selftest(uint64_t limit_ns, cudaStream_t stream, uint32_t* err);
 cudaError_t launch_gemv_direct(const GemvProblemDev* probs, int count, int batch, int N, int M,
                                cudaStream_t stream, int num_sms, uint32_t* err, bool dense2);
+// The dense 2-bit layout (also the codes plane of the 8:8 format) through
+// per-warp TMA rings (gemv_tma.cu).
+cudaError_t launch_gemv_dense_tma(const GemvProblemDev* probs, int count, int batch, cudaStream_t stream,
+                                  int num_sms, uint32_t* err);
 size_t dense2_row_bytes(int d_in);
 cudaError_t launch_pack_dense2(const int8_t* W_eff, int d_out, int d_in, uint8_t* out, cudaStream_t stream,
                                int num_sms);

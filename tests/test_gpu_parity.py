@@ -269,7 +269,7 @@ def test_pack_rejects_too_many_nonzeros(lib):
     lib.sbl_check()  # the latched error was cleared
 
 
-@pytest.fixture(params=[0, 1], ids=["direct", "ring"])
+@pytest.fixture(params=[0, 1, 2], ids=["stream", "ring", "direct"])
 def gemv_variant(request, lib):
     """Runs a GEMV test with each decode kernel (sbl_set_gemv_variant)."""
     lib.sbl_set_gemv_variant(request.param)

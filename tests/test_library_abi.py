@@ -100,7 +100,8 @@ def test_group_and_variant_validation_without_gpu(cl):
     al = 1 << 12
     assert cl.sbl_set_gemm_variant(2) == 1
     assert cl.sbl_set_gemm_variant(-1) == 1
-    assert cl.sbl_set_gemv_variant(2) == 1
+    assert cl.sbl_set_gemv_variant(3) == 1
+    assert cl.sbl_set_gemv_variant(-1) == 1
     assert cl.sbl_set_gemm_variant(0) == 0 and cl.sbl_set_gemv_variant(0) == 0
 
     def fwd(*problems):
