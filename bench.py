@@ -166,6 +166,22 @@ class Step:
         self.sparse24 = sparse24 and (N, M) == (2, 4)  # compress + sparse tensor-core forward
         self.kernels_per_step = 2 * n_p + n_x + 3 * n_p + (n_p if self.sparse24 else 0)
         self.train = False
+        self.pipelined = False
+
+    def enable_pipelined_weights(self):
+        """Compute the weight side (mask, gamma, ternary) of the next step
+        during this step's backward products, on the side streams, into a
+        second set of W_eff buffers; the step then starts with act_quant
+        alone.  The weight side is HBM-bound and the products are bound by
+        the tensor cores, so the two overlap.  Valid because W changes only
+        in an optimizer step, which the fwd + bwd step does not take (with
+        one, sbl_adamw_step computes the next weight side itself)."""
+        from semi_structured_sparsity_step_b200.layer import SparseBitLinearLayer
+        L0 = next(iter(self.layers.values()))
+        self.layers_next = {p.name: SparseBitLinearLayer(self.W[p.name], L0.N, L0.M, sparse24=self.sparse24)
+                            for p in self.ls.projections}
+        self.pipelined = True
+        self.primed = False
 
     def enable_training(self, lr=1e-5, betas=(0.9, 0.95), eps=1e-5, weight_decay=0.1, max_norm=1.0):
         """Make every step a full data-parallel training step: the dW of the
@@ -227,11 +243,31 @@ class Step:
                 join.record(sd)
                 stream.wait_event(join)
 
-        timed("weight_and_act_quant", weight_and_act_quant)
+        def act_quant_only():
+            for n, d in ls.inputs.items():
+                sbl.sbl_act_quant(self.X[n], T, d, self.Xq[n], self.amax[n], stream)
+
+        if self.pipelined:
+            if not self.primed:  # the first step computes its own weight side
+                weight_and_act_quant()
+                self.primed = True
+            else:
+                timed("act_quant", act_quant_only)
+        else:
+            timed("weight_and_act_quant", weight_and_act_quant)
         for p in ls.projections:
             L = self.layers[p.name]
             timed("forward_i8", lambda p=p, L=L: L.forward(self.Xq[p.input_name], self.amax[p.input_name],
                                                            self.Y[p.name], stream=stream))
+        if self.pipelined:
+            # the next step's weight side, overlapped with the backward products
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            for sd in self.side:
+                sd.wait_event(fork)
+            by_size = sorted(ls.projections, key=lambda p: -p.d_out * p.d_in)
+            for i, p in enumerate(by_size):
+                self.layers_next[p.name].weight_step(self.side[i % len(self.side)])
         for p in ls.projections:
             L = self.layers[p.name]
             timed("backward_dx_bf16", lambda p=p, L=L: L.backward(self.dY[p.name], self.X[p.input_name],
@@ -243,6 +279,12 @@ class Step:
                     self.exchange.launch(p.name)
         if self.train:
             timed("optimizer", lambda: self._optimizer(stream))
+        if self.pipelined:
+            for sd in self.side:
+                join = torch.cuda.Event()
+                join.record(sd)
+                stream.wait_event(join)
+            self.layers, self.layers_next = self.layers_next, self.layers
 
     def _optimizer(self, stream):
         """Wait for the dW exchange, then the global clip norm and AdamW with
@@ -874,6 +916,7 @@ def train_point(ls, T, N, M, sparse24, steps, warmup, X=None, dY=None, pk=None, 
         _, X, dY = make_inputs(ls, T, seed=0, device="cuda", with_weights=False)
     stream = torch.cuda.Stream()
     st = Step(ls, T, W, X, dY, N, M, sparse24)
+    st.enable_pipelined_weights()
     for _ in range(warmup):
         st.run(stream)
     stream.synchronize()
@@ -991,6 +1034,8 @@ def main():
     ap.add_argument("--sparse24", action="store_true", help="2:4: forward on the sparse tensor core")
     ap.add_argument("--settle-s", type=float, default=2.0,
                     help="untimed steps after the warm-up until this many seconds have passed")
+    ap.add_argument("--serial-weights", action="store_true",
+                    help="run each step's weight side before its forward instead of during the previous backward")
     ap.add_argument("--dp-train", action="store_true",
                     help="full data-parallel training step: dW summed over ranks (NCCL), clip norm, AdamW")
     ap.add_argument("--no-extras", action="store_true",
@@ -1024,11 +1069,15 @@ def main():
                           ", dY ~ N(0,1)",
               "tokens_per_step": T, "params": ls.params, "nm": f"{N_KEEP}:{M_GROUP}",
               "l2": "per-step working set larger than L2, no flush", "parallelism": f"dp{args.gpus} replicas",
+              "weight_side": "computed during the previous step's backward (pipelined)",
               "forward_kernel": ("2:4 compress + sparse int8 MMA (tcgen05.mma.sp)"
                                  if SPARSE24 and (N_KEEP, M_GROUP) == (2, 4)
                                  else "dense int8 MMA (tcgen05.mma kind::i8)")}
 
+    if args.serial_weights:
+        config["weight_side"] = "before the step's forward (overlapped with act_quant)"
     if args.dp_train:
+        config["weight_side"] = "fused into the optimizer step (sbl_adamw_step) of the previous step"
         config["parallelism"] = f"dp{args.gpus}: dW summed over ranks (NCCL all-reduce), then clip norm and AdamW"
         config["step"] = ("act quant, int8 forward, bf16 dX and dW, dW all-reduce per projection overlapping the "
                           "remaining products, sbl_grad_sqnorm, sbl_adamw_step with the next step's weight side")
@@ -1075,6 +1124,8 @@ def main():
         step = Step(ls, T, W, X, dY)
         if args.dp_train:
             step.enable_training()
+        elif not args.serial_weights:
+            step.enable_pipelined_weights()
     stream.synchronize()
 
     def barrier():
@@ -1142,6 +1193,8 @@ def main():
             st2 = Step(ls, T, W2, X2, dY2)
             if args.dp_train:
                 st2.enable_training()
+            elif not args.serial_weights:
+                st2.enable_pipelined_weights()
             sets.append((W2, X2, dY2, st2))
     outs_of = lambda st: [*st.Y.values(), *st.dX.values(), *st.dW.values()]  # noqa: E731
     host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs_of(st)] for (_, _, _, st) in sets]
