@@ -589,8 +589,9 @@ def run_decode(args):
             "workload": f"{layers} distinct qwen2.5-3b layer sets, packed {N_KEEP}:{M_GROUP} "
                         f"({'2.5 bit/weight' if (N_KEEP, M_GROUP) == (6, 8) else 'packed'}), "
                         f"batch 1/8/16, one grouped GEMV launch per layer (7 projections), CUDA graph per pass",
-            "gemv_kernel": ["streamed into fragments (small blocks)", "block-wide TMA ring",
-                            "per-warp TMA rings"][args.gemv_variant],
+            "gemv_kernel": ["dense layout: per-warp TMA rings filled before the dependency wait; "
+                            "N:M format: per-warp TMA rings in persistent blocks", "block-wide TMA ring",
+                            "per-warp TMA rings in persistent blocks"][args.gemv_variant],
             "peak_hbm_gbs": pkk["hbm"], "peak_source": pkk["src"], "results": results,
             "dense2": {"layout": "dense 2-bit codes of the same weights (2.0 bit/weight, no index plane)",
                        "results": results_d2}}
@@ -1029,7 +1030,7 @@ def main():
     ap.add_argument("--mode", choices=["train", "decode", "prefill", "normquant", "optimizer"], default="train")
     ap.add_argument("--layers", type=int, default=36, help="decode mode: distinct layer sets in the stack")
     ap.add_argument("--gemv-variant", type=int, default=0,
-                    help="decode kernel: 0 streamed into fragments (default), 1 block-wide TMA ring, 2 per-warp TMA rings")
+                    help="decode kernel: 0 default, 1 block-wide TMA ring, 2 per-warp TMA rings in persistent blocks")
     ap.add_argument("--nm", default="6:8", help="N:M of the mask (the sweep: 8:8, 6:8, 4:8, 2:8, 2:4)")
     ap.add_argument("--sparse24", action="store_true", help="2:4: forward on the sparse tensor core")
     ap.add_argument("--settle-s", type=float, default=2.0,
