@@ -76,8 +76,9 @@ int sbl_version(void);
  * all later calls in this process: 0 = pairs of CTAs computing 256 x 256
  * tiles with tcgen05 cta_group::2 (the default), 1 = one CTA per 128 x 256
  * tile.  Results are identical (integer forward) or differ only in fp32
- * summation order (backward).  Not a per-stream setting: do not change it
- * while calls are being enqueued from other threads. */
+ * summation order (backward).  A process-wide setting, not a per-stream
+ * one: safe to call from any thread (an atomic store); calls enqueued after
+ * it returns use the new kernel. */
 sbl_status sbl_set_gemm_variant(int variant);
 
 /* Select the decode GEMV kernel used by sbl_gemv_packed(_group) and
@@ -88,8 +89,8 @@ sbl_status sbl_set_gemm_variant(int variant);
  * block-wide TMA tile ring with producer and epilogue warps, 2 = persistent
  * blocks in which each warp streams its own 16-row slices through its own
  * TMA ring, for every format.  Results
- * are identical (exact int32 sums, the same scaling).  Same threading caveat
- * as sbl_set_gemm_variant. */
+ * are identical (exact int32 sums, the same scaling).  Process-wide and
+ * thread-safe like sbl_set_gemm_variant. */
 sbl_status sbl_set_gemv_variant(int variant);
 
 /* Failure-detection self-test.  Every spin-wait of this library gives up

@@ -27,6 +27,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -900,7 +901,7 @@ constexpr int kPackedStages = 4;
 // Which tensor-core kernel the products use: 0 = CTA pairs (default),
 // 1 = one CTA per 128 x 256 tile.  Process-wide; set through
 // sbl_set_gemm_variant().
-int g_gemm_variant = 0;
+std::atomic<int> g_gemm_variant{0};
 
 namespace {
 

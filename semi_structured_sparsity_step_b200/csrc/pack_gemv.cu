@@ -22,6 +22,7 @@
 // selected with sbl_set_gemv_variant(1); the default kernel, with a ring per
 // warp, is in gemv_direct.cu.  One launch serves a group of independent
 // problems (e.g. the seven projections of a layer).
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -607,18 +608,19 @@ cudaError_t launch_pack(const int8_t* W_eff, int d_out, int d_in, int N, int M, 
   return cudaGetLastError();
 }
 
-int g_gemv_variant = 0;
+std::atomic<int> g_gemv_variant{0};
 
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
                               cudaStream_t stream, int num_sms, uint32_t* err, bool dense2) {
   if (batch == 0 || count == 0) return cudaSuccess;
-  if (g_gemv_variant == 0 || g_gemv_variant == 2) {
+  const int variant = g_gemv_variant.load(std::memory_order_relaxed);
+  if (variant == 0 || variant == 2) {
     for (int c0 = 0; c0 < count; c0 += kGemvMaxGroup) {
       const int cnt = (count - c0) < kGemvMaxGroup ? (count - c0) : kGemvMaxGroup;
       // the dense layout (and the 8:8 format, whose codes plane it is) through
       // the TMA-fed kernel; the N:M formats through the per-warp ring kernel
       const bool dense = dense2 || N == M;
-      const cudaError_t e = (g_gemv_variant == 0 && dense)
+      const cudaError_t e = (variant == 0 && dense)
                                 ? launch_gemv_dense_tma(probs + c0, cnt, batch, stream, num_sms, err)
                                 : launch_gemv_direct(probs + c0, cnt, batch, N, M, stream, num_sms, err, dense2);
       if (e != cudaSuccess) return e;

@@ -2,6 +2,7 @@
 // (launchers called by the C ABI in sbl_api.cu).
 #pragma once
 
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
@@ -57,7 +58,7 @@ bool make_tmap_u32(CUtensorMap* m, const void* base, unsigned long long inner, u
 // Same for a uint8 matrix, with the 128-byte swizzle or none.
 bool make_tmap_u8(CUtensorMap* m, const void* base, unsigned long long inner, unsigned long long rows,
                   unsigned long long row_bytes, unsigned box_inner, unsigned box_rows, bool swizzle128);
-extern int g_gemm_variant;
+extern std::atomic<int> g_gemm_variant;
 cudaError_t launch_forward(const int8_t* Xq, const float* amax, const int8_t* W_eff, const float* gamma, int T,
                            int d_in, int d_out, float* Y, int32_t* acc, cudaStream_t stream, int num_sms,
                            uint32_t* err);
@@ -111,7 +112,7 @@ struct GemvProblemDev {
 // the N:M formats through gemv_direct.cu), 1 = block-wide TMA tile ring
 // (pack_gemv.cu), 2 = per-warp TMA rings in persistent blocks
 // (gemv_direct.cu) for every format.
-extern int g_gemv_variant;
+extern std::atomic<int> g_gemv_variant;
 cudaError_t launch_gemv_group(const GemvProblemDev* probs, int count, int batch, int N, int M,
                               cudaStream_t stream, int num_sms, uint32_t* err, bool dense2);
 // Failure-detection self-test: one bounded wait that runs out (selftest.cu).
