@@ -30,7 +30,8 @@
 // B = 112 rows x 256 bytes as two 128-byte swizzled column tiles, and the
 // 4096-byte selector block, all by TMA.  The MMA thread of the even CTA
 // copies the selectors into TMEM (tcgen05.cp, 128 lanes x 4 columns per
-// half; each instruction covers 64 weights = 2 columns) and issues four
+// half, into the 8 selector columns of that ring stage; each instruction
+// covers 64 weights = 2 columns) and issues four
 // M = 256, N = 224, K = 64 sparse MMAs.  Two 224-column accumulators in TMEM
 // let the epilogue of one tile overlap the next; the epilogue lane of weight
 // row o writes Y[t, o] for 32 tokens at a time, so each store instruction of
@@ -57,12 +58,12 @@ constexpr int kSpStageBytes = kSpABytes + kSpBBytes + kSpEBytes;
 constexpr int kSpSmem = kSpStages * kSpStageBytes + 1024 + 256;
 constexpr int kSpThreads = 192;
 constexpr uint32_t kSpTmemCols = 512;
-constexpr uint32_t kSpECol = 2 * kSpBN;     // selector columns after the two accumulators
+constexpr uint32_t kSpECol = 2 * kSpBN;     // selector columns after the two accumulators, 8 per ring stage
 constexpr uint32_t kSpIdesc = instr_desc(true, 256, kSpBN, false, false) | (1u << 2);  // bit 2: sparse A
 
 static_assert(kSpStageBytes % 1024 == 0, "stage bases stay 1024-byte aligned");
 static_assert((kSpABytes + kSpBTile) % 1024 == 0, "second B tile is 1024-byte aligned");
-static_assert(kSpECol + 8 <= kSpTmemCols, "selectors fit after the accumulators");
+static_assert(kSpECol + 8 * kSpStages <= kSpTmemCols, "every stage's selectors fit after the accumulators");
 
 struct Sp24Args {
   int T, d_in, d_out;
@@ -165,7 +166,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSpThreads, 1)
     if (lane == 0 && leader) {
       int it = 0, t = 0;
       bool ok = true;
-      const uint32_t e_tmem = tmem_base + kSpECol;
       for (int w = pair_id; w < args.total && ok; w += n_pairs, ++t) {
         const int b = t & 1;
         if (!mbar_wait(&tempty[b], (static_cast<uint32_t>(t >> 1) & 1u) ^ 1u, abort_flag, args.err)) {
@@ -186,6 +186,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSpThreads, 1)
           const uint32_t sa = smem_u32(smem + s * kSpStageBytes);
           const uint32_t sb = sa + kSpABytes;
           const uint32_t se = sb + kSpBBytes;
+          // each ring stage has its own selector columns, so copying the next
+          // stage's selectors never waits for this stage's products to read theirs
+          const uint32_t e_tmem = tmem_base + kSpECol + 8u * static_cast<uint32_t>(s);
           pair::tmem_cp_128x128b(e_tmem, smem_desc_rows16(se, 128));
           pair::tmem_cp_128x128b(e_tmem + 4, smem_desc_rows16(se + 2048, 128));
 #pragma unroll
