@@ -589,7 +589,7 @@ def run_decode(args):
             "workload": f"{layers} distinct qwen2.5-3b layer sets, packed {N_KEEP}:{M_GROUP} "
                         f"({'2.5 bit/weight' if (N_KEEP, M_GROUP) == (6, 8) else 'packed'}), "
                         f"batch 1/8/16, one grouped GEMV launch per layer (7 projections), CUDA graph per pass",
-            "gemv_kernel": ["dense layout: per-warp TMA rings filled before the dependency wait; "
+            "gemv_kernel": ["dense layout: per-warp TMA rings filled before the dependency wait, activations staged in shared memory; "
                             "N:M format: per-warp TMA rings in persistent blocks", "block-wide TMA ring",
                             "per-warp TMA rings in persistent blocks"][args.gemv_variant],
             "peak_hbm_gbs": pkk["hbm"], "peak_source": pkk["src"], "results": results,
