@@ -50,7 +50,7 @@ WORKLOADS = {
     "qwen2.5-3b-up": (8192, "trimodal", 0.001, 0.01),
 }
 N_KEEP, M_GROUP = 6, 8
-SPARSE24 = False  # --sparse24: 2:4 layers use the sparse tensor core
+SPARSE24 = True  # 2:4 layers use the sparse tensor core (--dense24: the dense int8 product)
 METRIC = "Sparse-BitLinear fwd+bwd tokens/s (3B-shape, 6:8)"
 
 NOMINAL_I8_OVER_BF16 = 2.0  # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
@@ -1032,7 +1032,9 @@ def main():
     ap.add_argument("--gemv-variant", type=int, default=0,
                     help="decode kernel: 0 default, 1 block-wide TMA ring, 2 per-warp TMA rings in persistent blocks")
     ap.add_argument("--nm", default="6:8", help="N:M of the mask (the sweep: 8:8, 6:8, 4:8, 2:8, 2:4)")
-    ap.add_argument("--sparse24", action="store_true", help="2:4: forward on the sparse tensor core")
+    ap.add_argument("--sparse24", action="store_true",
+                    help="2:4: forward on the sparse tensor core (the default; kept for explicit commands)")
+    ap.add_argument("--dense24", action="store_true", help="2:4: forward through the dense int8 product instead")
     ap.add_argument("--settle-s", type=float, default=2.0,
                     help="untimed steps after the warm-up until this many seconds have passed")
     ap.add_argument("--serial-weights", action="store_true",
@@ -1044,7 +1046,7 @@ def main():
     args = ap.parse_args()
     global N_KEEP, M_GROUP, SPARSE24
     N_KEEP, M_GROUP = (int(v) for v in args.nm.split(":"))
-    SPARSE24 = args.sparse24
+    SPARSE24 = not args.dense24
     if args.mode == "decode":
         print(json.dumps(run_decode(args)))
         return

@@ -33,9 +33,12 @@
 // half, into the 8 selector columns of that ring stage; each instruction
 // covers 64 weights = 2 columns) and issues four
 // M = 256, N = 224, K = 64 sparse MMAs.  Two 224-column accumulators in TMEM
-// let the epilogue of one tile overlap the next; the epilogue lane of weight
-// row o writes Y[t, o] for 32 tokens at a time, so each store instruction of
-// a warp covers 32 consecutive floats of a Y row.
+// let the epilogue of one tile overlap the next.  The epilogue reads each
+// 32 x 32 chunk with one weight row per lane and turns it around in a padded
+// shared tile, so that every 16-byte store of a warp lands in one of four
+// whole 128-byte segments of Y rows (the epilogue, not the tensor core, is
+// what bounds this kernel: the MMA thread waited half its time for a free
+// accumulator with one 4-byte store per lane and token).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -55,7 +58,9 @@ constexpr int kSpBTile = kSpHalfN * 128;    // one 128-byte column tile of B
 constexpr int kSpBBytes = 2 * kSpBTile;
 constexpr int kSpEBytes = 4096;             // selector block
 constexpr int kSpStageBytes = kSpABytes + kSpBBytes + kSpEBytes;
-constexpr int kSpSmem = kSpStages * kSpStageBytes + 1024 + 256;
+constexpr int kSpEpiStride = 36;            // floats per row of an epilogue warp's 32 x 32 transpose tile
+constexpr int kSpEpiBytes = 4 * 32 * kSpEpiStride * 4;
+constexpr int kSpSmem = kSpStages * kSpStageBytes + 256 + kSpEpiBytes + 1024;
 constexpr int kSpThreads = 192;
 constexpr uint32_t kSpTmemCols = 512;
 constexpr uint32_t kSpECol = 2 * kSpBN;     // selector columns after the two accumulators, 8 per ring stage
@@ -87,6 +92,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSpThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* epi_tiles = reinterpret_cast<uint32_t*>(smem + kSpStages * kSpStageBytes + 256);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -226,9 +232,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSpThreads, 1)
       }
       tc_fence_after();
       if (*abort_flag) break;
-      const int o = mb * 256 + 128 * static_cast<int>(rank) + 32 * q + lane;
-      const bool row_ok = o < args.d_out;
+      // Each 32 x 32 chunk (lane = weight row, register j = token) goes through
+      // a padded shared tile so that the stores run along Y's rows: lane l then
+      // holds rows o0 + 4 (l % 8) .. + 3 of token 4 it + l / 8, one 16-byte
+      // store per lane and four whole 128-byte row segments per instruction.
+      const int o0 = mb * 256 + 128 * static_cast<int>(rank) + 32 * q;  // the warp's first weight row
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b * kSpBN);
+      uint32_t* et = epi_tiles + (warp - 2) * (32 * kSpEpiStride);
+      const int c4 = 4 * (lane & 7), tr = lane >> 3;
+      const bool cols_ok = o0 + c4 < args.d_out;  // d_out % 8 == 0: four rows are all in or all out
 #pragma unroll
       for (int c = 0; c < kSpBN / 32; ++c) {
         const int t0 = nb * kSpBN + 32 * c;
@@ -236,20 +248,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSpThreads, 1)
         uint32_t r[32];
         tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(32 * c), r);
         tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) et[j * kSpEpiStride + lane] = r[j];
+        __syncwarp();
         const float sl = scl[c];
-        float* yc = args.Y + static_cast<long long>(t0) * args.d_out + o;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float sj = __shfl_sync(0xFFFFFFFFu, sl, j);
-          if (row_ok && t0 + j < args.T)
-            yc[static_cast<long long>(j) * args.d_out] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), sj);
+        for (int it = 0; it < 8; ++it) {
+          const int tl = 4 * it + tr;  // token within the chunk
+          const float sc = __shfl_sync(0xFFFFFFFFu, sl, tl);
+          const uint4 v = *reinterpret_cast<const uint4*>(et + tl * kSpEpiStride + c4);
+          if (cols_ok && t0 + tl < args.T) {
+            const long long off = static_cast<long long>(t0 + tl) * args.d_out + o0 + c4;
+            *reinterpret_cast<float4*>(args.Y + off) =
+                make_float4(__fmul_rn(__int2float_rn(static_cast<int>(v.x)), sc),
+                            __fmul_rn(__int2float_rn(static_cast<int>(v.y)), sc),
+                            __fmul_rn(__int2float_rn(static_cast<int>(v.z)), sc),
+                            __fmul_rn(__int2float_rn(static_cast<int>(v.w)), sc));
+            if (args.acc != nullptr) *reinterpret_cast<uint4*>(args.acc + off) = v;
+          }
         }
-        if (args.acc != nullptr && row_ok) {
-          int32_t* ac = args.acc + static_cast<long long>(t0) * args.d_out + o;
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (t0 + j < args.T) ac[static_cast<long long>(j) * args.d_out] = static_cast<int32_t>(r[j]);
-        }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
