@@ -482,6 +482,39 @@ def test_gemv_dense2_group_matches_oracle(lib, gemv_variant, batch):
         assert np.array_equal(Y.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("batch", [1, 2, 8])
+def test_gemv_dense2_group_shared_activations(lib, batch):
+    """Projections that read the same activations (as q, k and v do) in one
+    grouped launch: the kernel stages each activation tensor in shared memory
+    once per block when it fits and shares it between those problems, and
+    reads the rest (here the 11008-wide input at batch > 1) from global
+    memory; every output must still be the oracle's, bit for bit."""
+    inputs = {"a": 2048, "b": 11008, "c": 4864}
+    shapes = [("a", 264), ("a", 40), ("a", 1040), ("b", 136), ("c", 520), ("c", 8)]
+    xs = {}
+    for j, (name, d_in) in enumerate(inputs.items()):
+        x = synth.activations(batch, d_in, seed=84, tensor_id=100 + j)
+        xq, amax = oracle.act_quant(synth.bits(x))
+        xs[name] = (xq, amax, torch.from_numpy(xq).cuda(), torch.from_numpy(amax).cuda())
+    probs, refs = [], []
+    for i, (name, d_out) in enumerate(shapes):
+        d_in = inputs[name]
+        w = synth.trimodal_weight(d_out, d_in, seed=84, tensor_id=i)
+        weff, gamma, _ = oracle.effective_weight(synth.bits(w), 6, 8)
+        nbytes = lib.sbl_dense2_bytes(d_out, d_in)
+        d2 = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        lib.sbl_pack_dense2(torch.from_numpy(weff).cuda(), d_out, d_in, d2, nbytes)
+        Y = torch.full((batch, d_out), float("nan"), dtype=torch.float32, device="cuda")
+        g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+        xq, amax, xq_d, amax_d = xs[name]
+        probs.append((d2, xq_d, amax_d, g, Y, d_in, d_out))
+        refs.append(oracle.forward_out(oracle.forward_acc(xq, weff), gamma, amax))
+    lib.sbl_gemv_dense2_group(probs, batch)
+    lib.sbl_check()
+    for (_, _, _, _, Y, _, _), ref in zip(probs, refs):
+        assert np.array_equal(Y.cpu().numpy(), ref)
+
+
 @pytest.mark.parametrize("N,M", [(1, 8), (3, 8), (5, 8), (7, 8), (1, 4), (3, 4), (4, 8)])
 @pytest.mark.parametrize("d_out,d_in", [(8, 16), (24, 48), (40, 2320), (136, 4368)])
 def test_gemv_every_k_and_ragged_rows(lib, gemv_variant, N, M, d_out, d_in):
