@@ -306,22 +306,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     lrbs.n = l;
     // Activations of the block's problems go to shared memory while they
     // fit, in order; problems that read the same activations share a copy.
-    int used = 0;
+    long long used = 0;
     for (int i = 0; i < kMaxGroup; ++i) xoff[i] = -1, xown[i] = 0;
     if (l > 0) {
       for (int q = lrbs.pi[0]; q <= lrbs.pi[l - 1]; ++q) {
         const DenseProblem& P = grp.p[q];
         for (int e = lrbs.pi[0]; e < q; ++e)
           if (xoff[e] >= 0 && grp.p[e].Xq == P.Xq && grp.p[e].d_in == P.d_in) xoff[q] = xoff[e];
-        const int bytes = batch * P.d_in;
+        const long long bytes = static_cast<long long>(batch) * P.d_in;
         if (xoff[q] < 0 && used + bytes <= grp.xbytes) {
-          xoff[q] = used;
+          xoff[q] = static_cast<int>(used);
           xown[q] = 1;
           used += bytes;
         }
       }
     }
-    xtotal = used;
+    xtotal = static_cast<int>(used);  // at most grp.xbytes
   }
   for (int i = threadIdx.x; i < kMaxLocalRB * 16 * batch; i += kThreads) accum[i] = 0;
   __syncthreads();
